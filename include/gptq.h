@@ -1,0 +1,172 @@
+/*
+ * gptq.h - C ABI of a B200 (sm_100a) library for GPTQ post-training weight
+ * quantization of one linear layer.
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ * - All tensors are dense, row-major and in caller-owned DEVICE memory on the
+ *   current CUDA device.  The library never frees or retains a caller
+ *   pointer.  Device pointers must be 16-byte aligned.
+ * - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   Work is enqueued on that stream in order.
+ * - The return value is a gptq_status.  Arguments are validated on the host
+ *   before any work is enqueued; a rejected call changes no output.
+ * - Notation: W is [n_out, n_in] (a torch.nn.Linear weight), X is
+ *   [tokens, n_in] calibration activations, H = 2 X^T X is [n_in, n_in].
+ *
+ * Sources of the operations (page title and section):
+ * - "第5章 GPTQ 实战：如何把 Hugging Face 模型量化成 4-bit" (CSDN, chapter 5):
+ *   §5.1.4 objective ||(W - W_q) X||^2; §5.1.7 Hessian H = X X^T up to a
+ *   constant; §5.1.8 damping, Cholesky of the inverse, quantize-and-compensate
+ *   sweep with lazy block updates; §5.1.10 group-wise scales.
+ * - "AutoGPTQ 官方示例全解析" §1.4 and "OLMo 仓库中的 AutoGPTQ 快速上手" §三:
+ *   BaseQuantizeConfig fields bits / group_size / damp_percent / desc_act /
+ *   static_groups / sym and their validity rules.
+ */
+#ifndef GPTQ_H
+#define GPTQ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GPTQ_OK = 0,
+  GPTQ_ERR_INVALID_ARG = 1, /* value outside what the config rules allow (ValueError analogue) */
+  GPTQ_ERR_UNSUPPORTED = 2, /* valid per the pages but not handled by this library (sizes, alignment) */
+  GPTQ_ERR_NOT_PD = 3,      /* damped Hessian has a non-positive or non-finite pivot */
+  GPTQ_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
+  GPTQ_ERR_OOM = 5,         /* workspace allocation failed */
+  GPTQ_ERR_TIMEOUT = 6      /* a bounded device-side wait gave up */
+} gptq_status;
+
+typedef enum { GPTQ_F32 = 0, GPTQ_F16 = 1, GPTQ_BF16 = 2 } gptq_dtype;
+
+/* Optional per-call report of gptq_quantize_layer / _factored. */
+typedef struct {
+  double damped_loss;  /* sum over rows and columns of err^2, err = (w - w_hat) / U_jj */
+  float ms_prepare;    /* act-order permutation, damping copy, weight staging, fixed group params */
+  float ms_factor;     /* damped Cholesky and triangular inverse (0 for the _factored call) */
+  float ms_sweep;      /* quantize-and-compensate sweep including lazy updates */
+  float ms_pack;       /* code packing and g_idx */
+  int32_t panel_width; /* columns per sweep panel chosen by the library */
+  int32_t outer_width; /* columns per lazy-update block chosen by the library */
+} gptq_stats;
+
+/*
+ * H += 2 * X^T X.
+ * Source: chapter 5 §5.1.7 (the layer's reconstruction Hessian is X X^T up to
+ * a constant, estimated from calibration data); with tokens as rows of X the
+ * product is X^T X, and the constant 2 is the Hessian of the squared error.
+ *
+ * X       [tokens, n_in] fp16 (x_dtype = GPTQ_F16) or bf16 (GPTQ_BF16), read-only.
+ * tokens  >= 0; tokens == 0 is a no-op.
+ * n_in    > 0; must be a multiple of 8 (16-byte rows for TMA), else UNSUPPORTED.
+ * H       [n_in, n_in] fp32, read-modify-write.  Both triangles are written.
+ *         The caller zero-initialises H once; repeated calls over chunks of
+ *         tokens accumulate (streaming calibration).  Products are exact in
+ *         fp32; sums are fp32 with periodic re-normalisation of the
+ *         tensor-core accumulator (relative Frobenius error <= 1e-5).
+ * Asynchronous on `stream`: only host-detectable errors are returned.  A
+ * device-side timeout is recorded and reported by gptq_device_status().
+ */
+int gptq_accumulate_hessian(const void* X, int x_dtype, int64_t tokens, int64_t n_in,
+                            float* H, void* stream);
+
+/*
+ * Quantize one linear layer with GPTQ.
+ * Source: chapter 5 §5.1.8 (damping H + damp*mean(diag H)*I, one Cholesky of
+ * the inverse, column sweep: quantize with the group's fixed scale, normalise
+ * the error by the factor's diagonal, subtract it times the factor row from the
+ * later columns, lazily per block), §5.1.10 (group-wise scales); config rules
+ * from the AutoGPTQ examples guide §1.4.
+ *
+ * W          [n_out, n_in] fp32/fp16/bf16 (w_dtype), read-only.
+ * H          [n_in, n_in] fp32 symmetric calibration Hessian, read-only (it may be
+ *            shared by several layers that see the same input).
+ * bits       2, 3, 4 or 8, else INVALID_ARG.
+ * group_size -1 (one group per output row, parameters from the row before any
+ *            update) or > 0 dividing n_in; 0, < -1 or not dividing -> INVALID_ARG.
+ * damp_percent in (0, 1), else (or NaN) INVALID_ARG.
+ * sym        nonzero: s = 2 max|x| / maxq, zero = 2^(bits-1);
+ *            zero: range [min(0,min x), max(0,max x)], zero = rint(-lo/s).
+ * desc_act   nonzero: columns are processed in order of descending diag(H)
+ *            (stable for ties).
+ * static_groups nonzero (with group_size > 0): every group's parameters come
+ *            from the original W before any update; column c uses group c/group_size.
+ *            Otherwise a group's parameters come from the current, already
+ *            error-updated weights when the sweep reaches its first column.
+ * blocksize  > 0, else INVALID_ARG.  The lazy-update block width; results do
+ *            not depend on it beyond floating-point rounding, and the library
+ *            may choose a different internal panel width aligned to groups.
+ * Outputs (device, written completely on GPTQ_OK):
+ *   qweight [n_in*bits/32, n_out] int32: for each output channel o the codes
+ *           along n_in (original column order) form an LSB-first stream of
+ *           bits-wide fields cut into 32-bit words (3-bit fields straddle words).
+ *   scales  [G, n_out] fp32, zeros [G, n_out] int32 in [0, 2^bits - 1],
+ *           G = n_in / group_size (1 if group_size == -1).
+ *   g_idx   [n_in] int32: group of each original input column.
+ *   Dequantized weight: scales[g_idx[c], o] * (code[o, c] - zeros[g_idx[c], o]).
+ * n_in*bits % 32 != 0 or n_in % 8 != 0 -> UNSUPPORTED.
+ * Workspace (about 2*n_in^2*4 + n_out*n_in*5 bytes) is allocated stream-ordered
+ * inside the call (OOM if that fails).  The call is blocking: it synchronises
+ * `stream` once at the end and returns NOT_PD if a pivot failed.
+ * stats may be NULL.
+ */
+int gptq_quantize_layer(const void* W, int w_dtype, int64_t n_out, int64_t n_in,
+                        const float* H, int bits, int group_size, float damp_percent,
+                        int sym, int desc_act, int static_groups, int blocksize,
+                        int32_t* qweight, float* scales, int32_t* zeros, int32_t* g_idx,
+                        void* stream, gptq_stats* stats);
+
+/*
+ * The factor half of gptq_quantize_layer, for layers that share one Hessian
+ * (q/k/v, gate/up): factor once, sweep many.
+ * Source: chapter 5 §5.1.8, damping and "Cholesky(inverse(H))".
+ *
+ * H     [n_in, n_in] fp32 symmetric, read-only.
+ * U     [n_in, n_in] fp32 output: upper-triangular factor, in sweep order, of
+ *       the inverse of the damped (and, with desc_act, permuted) Hessian:
+ *       inverse(H_d) = U^T U, U_jj > 0.  The strictly lower triangle is zero.
+ * perm  [n_in] int32 output: sweep position j processes original column perm[j]
+ *       (identity without desc_act).
+ * Blocking; returns NOT_PD on a failed pivot.  UNSUPPORTED if n_in % 8 != 0.
+ */
+int gptq_factor_hessian(const float* H, int64_t n_in, float damp_percent, int desc_act,
+                        float* U, int32_t* perm, void* stream);
+
+/*
+ * The sweep half: quantize W given the factor U and permutation perm produced
+ * by gptq_factor_hessian (or any upper-triangular U with positive diagonal).
+ * Arguments and outputs as in gptq_quantize_layer; U and perm are read-only.
+ * Blocking.
+ */
+int gptq_quantize_layer_factored(const void* W, int w_dtype, int64_t n_out, int64_t n_in,
+                                 const float* U, const int32_t* perm, int bits, int group_size,
+                                 int sym, int static_groups, int blocksize,
+                                 int32_t* qweight, float* scales, int32_t* zeros,
+                                 int32_t* g_idx, void* stream, gptq_stats* stats);
+
+/*
+ * Synchronise `stream` and return the library's asynchronous device status
+ * (GPTQ_OK or GPTQ_ERR_TIMEOUT from a bounded wait in an asynchronous call).
+ * clear != 0 resets it to GPTQ_OK afterwards.
+ */
+int gptq_device_status(void* stream, int clear);
+
+/* Static description of a status code (never NULL). */
+const char* gptq_status_string(int status);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t gptq_launch_count(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int gptq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPTQ_H */

@@ -1,0 +1,135 @@
+"""Torch-facing wrappers of the C ABI (argument marshalling only).
+
+Tensors must already live on a CUDA device; outputs are allocated with torch
+(device memory plumbing) and filled by the native kernels.  Every call goes to
+``lib/libgptq.so``; nothing here computes any part of the method.
+"""
+
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from ._native import GptqStats, lib
+
+OK, INVALID_ARG, UNSUPPORTED, NOT_PD, CUDA_ERR, OOM, TIMEOUT = range(7)
+_DTYPE = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
+
+
+class GPTQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib().gptq_status_string(status).decode()
+        super().__init__(f"{where}: {msg} (status {status})")
+
+
+def _check(st, where):
+    if st != OK:
+        raise GPTQError(st, where)
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if not (isinstance(t, torch.Tensor) and t.is_cuda):
+            raise ValueError("tensors must be CUDA tensors")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def group_count(n_in: int, group_size: int) -> int:
+    return 1 if group_size == -1 else n_in // group_size
+
+
+@dataclass
+class QuantResult:
+    qweight: torch.Tensor
+    scales: torch.Tensor
+    zeros: torch.Tensor
+    g_idx: torch.Tensor
+    stats: dict | None = None
+
+
+def accumulate_hessian(X: torch.Tensor, H: torch.Tensor, stream=None) -> torch.Tensor:
+    """H += 2 X^T X (asynchronous on the stream).  X [T, n] fp16/bf16, H [n, n] fp32."""
+    _need_cuda(X, H)
+    if X.dim() != 2 or H.shape != (X.shape[1], X.shape[1]) or H.dtype != torch.float32:
+        raise ValueError("X must be [tokens, n_in] and H [n_in, n_in] float32")
+    st = lib().gptq_accumulate_hessian(_ptr(X), _DTYPE.get(X.dtype, 99), X.shape[0], X.shape[1], _ptr(H),
+                                       _stream(stream))
+    _check(st, "gptq_accumulate_hessian")
+    return H
+
+
+def device_status(clear: bool = True, stream=None) -> int:
+    return lib().gptq_device_status(_stream(stream), 1 if clear else 0)
+
+
+def launch_count() -> int:
+    return lib().gptq_launch_count()
+
+
+def _outputs(n_out, n_in, bits, group_size, device, out):
+    if out is not None:
+        return out
+    G = group_count(n_in, group_size)
+    return (torch.empty(n_in * bits // 32, n_out, dtype=torch.int32, device=device),
+            torch.empty(G, n_out, dtype=torch.float32, device=device),
+            torch.empty(G, n_out, dtype=torch.int32, device=device),
+            torch.empty(n_in, dtype=torch.int32, device=device))
+
+
+def _stats_dict(s: GptqStats):
+    return {k: getattr(s, k) for k, _ in GptqStats._fields_}
+
+
+def quantize_layer(W, H, bits=4, group_size=128, damp_percent=0.01, sym=True, desc_act=False,
+                   static_groups=False, blocksize=128, stats=False, out=None, stream=None) -> QuantResult:
+    """GPTQ of one linear layer: W [n_out, n_in] (fp32/fp16/bf16), H [n_in, n_in] fp32."""
+    _need_cuda(W, H)
+    n_out, n_in = W.shape
+    qw, sc, zr, gi = _outputs(n_out, n_in, bits, group_size, W.device, out)
+    st_obj = GptqStats() if stats else None
+    st = lib().gptq_quantize_layer(
+        _ptr(W), _DTYPE.get(W.dtype, 99), n_out, n_in, _ptr(H), bits, group_size, float(damp_percent),
+        int(bool(sym)), int(bool(desc_act)), int(bool(static_groups)), blocksize, _ptr(qw), _ptr(sc),
+        _ptr(zr), _ptr(gi), _stream(stream), ctypes.byref(st_obj) if stats else None)
+    _check(st, "gptq_quantize_layer")
+    return QuantResult(qw, sc, zr, gi, _stats_dict(st_obj) if stats else None)
+
+
+def factor_hessian(H, damp_percent=0.01, desc_act=False, stream=None):
+    """Returns (U, perm): inverse(H_d) = U^T U in sweep order, perm = column order."""
+    _need_cuda(H)
+    n = H.shape[0]
+    U = torch.empty(n, n, dtype=torch.float32, device=H.device)
+    perm = torch.empty(n, dtype=torch.int32, device=H.device)
+    st = lib().gptq_factor_hessian(_ptr(H), n, float(damp_percent), int(bool(desc_act)), _ptr(U), _ptr(perm),
+                                   _stream(stream))
+    _check(st, "gptq_factor_hessian")
+    return U, perm
+
+
+def quantize_layer_factored(W, U, perm, bits=4, group_size=128, sym=True, static_groups=False, blocksize=128,
+                            stats=False, out=None, stream=None) -> QuantResult:
+    _need_cuda(W, U, perm)
+    n_out, n_in = W.shape
+    qw, sc, zr, gi = _outputs(n_out, n_in, bits, group_size, W.device, out)
+    st_obj = GptqStats() if stats else None
+    st = lib().gptq_quantize_layer_factored(
+        _ptr(W), _DTYPE.get(W.dtype, 99), n_out, n_in, _ptr(U), _ptr(perm), bits, group_size, int(bool(sym)),
+        int(bool(static_groups)), blocksize, _ptr(qw), _ptr(sc), _ptr(zr), _ptr(gi), _stream(stream),
+        ctypes.byref(st_obj) if stats else None)
+    _check(st, "gptq_quantize_layer_factored")
+    return QuantResult(qw, sc, zr, gi, _stats_dict(st_obj) if stats else None)

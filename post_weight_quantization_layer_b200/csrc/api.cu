@@ -1,0 +1,299 @@
+// extern "C" entry points: argument validation, workspace, orchestration, status.
+#include <cmath>
+#include <cstring>
+
+#include "common.cuh"
+
+namespace gptq {
+
+std::atomic<uint64_t> g_launches{0};
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+
+// Stream-ordered workspace: one allocation carved into aligned pieces.
+struct Workspace {
+  char* base = nullptr;
+  size_t used = 0;
+  size_t cap = 0;
+  cudaStream_t s = nullptr;
+  ~Workspace() {
+    if (base) cudaFreeAsync(base, s);
+  }
+  template <typename T>
+  T* take(size_t count) {
+    const size_t off = (used + 255) & ~size_t(255);
+    used = off + count * sizeof(T);
+    return reinterpret_cast<T*>(base + off);
+  }
+};
+
+size_t padded(size_t bytes) { return (bytes + 255) & ~size_t(255); }
+
+int alloc(Workspace& ws, size_t bytes, cudaStream_t s) {
+  ws.s = s;
+  ws.cap = bytes;
+  cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&ws.base), bytes, s);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    ws.base = nullptr;
+    return GPTQ_ERR_OOM;
+  }
+  return GPTQ_OK;
+}
+
+// Read the device status word after the stream drains.
+int finish(int* dstatus, cudaStream_t s) {
+  int h = 0;
+  if (cudaMemcpyAsync(&h, dstatus, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess) return GPTQ_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return GPTQ_ERR_CUDA;
+  return h;
+}
+
+bool valid_damp(float d) { return d > 0.f && d < 1.f; }  // false for NaN
+
+int check_quant_args(const void* W, int w_dtype, int64_t n_out, int64_t n_in, int bits, int group_size,
+                     int blocksize, const void* qweight, const void* scales, const void* zeros, const void* g_idx) {
+  if (!W || !qweight || !scales || !zeros || !g_idx) return GPTQ_ERR_INVALID_ARG;
+  if (w_dtype != GPTQ_F32 && w_dtype != GPTQ_F16 && w_dtype != GPTQ_BF16) return GPTQ_ERR_INVALID_ARG;
+  if (n_out <= 0 || n_in <= 0) return GPTQ_ERR_INVALID_ARG;
+  if (bits != 2 && bits != 3 && bits != 4 && bits != 8) return GPTQ_ERR_INVALID_ARG;
+  if (!(group_size == -1 || group_size > 0)) return GPTQ_ERR_INVALID_ARG;
+  if (group_size > 0 && n_in % group_size != 0) return GPTQ_ERR_INVALID_ARG;
+  if (blocksize <= 0) return GPTQ_ERR_INVALID_ARG;
+  if (n_in % 8 != 0 || (n_in * bits) % 32 != 0) return GPTQ_ERR_UNSUPPORTED;
+  if (n_in > 65535 || n_out > 65535) return GPTQ_ERR_UNSUPPORTED;
+  if (!aligned16(W) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) || !aligned16(g_idx))
+    return GPTQ_ERR_UNSUPPORTED;
+  return GPTQ_OK;
+}
+
+__global__ void invert_perm_kernel(const int32_t* __restrict__ perm, int64_t n, int32_t* __restrict__ invperm,
+                                   int* status) {
+  const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (j >= n) return;
+  const int32_t p = perm[j];
+  if (p < 0 || p >= n) {
+    atomicExch(status, GPTQ_ERR_INVALID_ARG);
+    return;
+  }
+  invperm[p] = static_cast<int32_t>(j);
+}
+
+__global__ void iota_kernel(int32_t* __restrict__ p, int64_t n) {
+  const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (j < n) p[j] = static_cast<int32_t>(j);
+}
+
+// A permutation is valid iff invperm[perm[j]] == j for every j (after the scatter).
+__global__ void check_perm_kernel(const int32_t* __restrict__ perm, const int32_t* __restrict__ invperm, int64_t n,
+                                  int* status) {
+  const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (j >= n) return;
+  const int32_t p = perm[j];
+  if (p < 0 || p >= n || invperm[p] != j) atomicExch(status, GPTQ_ERR_INVALID_ARG);
+}
+
+struct Events {
+  cudaEvent_t ev[6] = {};
+  bool on = false;
+  int create(bool want) {
+    on = want;
+    if (!on) return GPTQ_OK;
+    for (auto& e : ev)
+      if (cudaEventCreate(&e) != cudaSuccess) return GPTQ_ERR_CUDA;
+    return GPTQ_OK;
+  }
+  ~Events() {
+    if (on)
+      for (auto& e : ev)
+        if (e) cudaEventDestroy(e);
+  }
+  float ms(int a, int b) {
+    float t = 0.f;
+    if (on) cudaEventElapsedTime(&t, ev[a], ev[b]);
+    return t;
+  }
+};
+
+int sweep_common(const void* W, int w_dtype, int64_t n_out, int64_t n_in, const float* U, const int32_t* perm,
+                 const int32_t* invperm, int bits, int group_size, int sym, int static_groups, int blocksize,
+                 int32_t* qweight, float* scales, int32_t* zeros, int32_t* g_idx, float* Wk, uint8_t* codesT,
+                 double* loss, int* status, cudaStream_t s, gptq_stats* stats, Events& evs, int ev0) {
+  SweepArgs a;
+  a.W = W;
+  a.w_dtype = w_dtype;
+  a.n_out = n_out;
+  a.n_in = n_in;
+  a.U = U;
+  a.perm = perm;
+  a.invperm = invperm;
+  a.bits = bits;
+  a.group_size = group_size;
+  a.sym = sym != 0;
+  a.static_groups = static_groups != 0 && group_size > 0;
+  a.blocksize = blocksize;
+  a.qweight = qweight;
+  a.scales = scales;
+  a.zeros = zeros;
+  a.g_idx = g_idx;
+  a.Wk = Wk;
+  a.codesT = codesT;
+  a.loss = loss;
+  a.status = status;
+  a.stats = stats;
+  for (int i = 0; i < 4; ++i) a.ev[i] = evs.on ? evs.ev[ev0 + i] : nullptr;
+  int pw = 0, qw = 0;
+  GPTQ_TRY(run_sweep(a, s, &pw, &qw));
+  if (stats) {
+    stats->panel_width = pw;
+    stats->outer_width = qw;
+  }
+  return GPTQ_OK;
+}
+
+}  // namespace
+}  // namespace gptq
+
+using namespace gptq;
+
+extern "C" {
+
+int gptq_version(void) { return kVersion; }
+
+uint64_t gptq_launch_count(void) { return g_launches.load(); }
+
+const char* gptq_status_string(int status) {
+  switch (status) {
+    case GPTQ_OK: return "ok";
+    case GPTQ_ERR_INVALID_ARG: return "invalid argument";
+    case GPTQ_ERR_UNSUPPORTED: return "unsupported size, dtype or alignment";
+    case GPTQ_ERR_NOT_PD: return "damped Hessian is not positive definite";
+    case GPTQ_ERR_CUDA: return "CUDA error";
+    case GPTQ_ERR_OOM: return "workspace allocation failed";
+    case GPTQ_ERR_TIMEOUT: return "bounded device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int gptq_accumulate_hessian(const void* X, int x_dtype, int64_t tokens, int64_t n_in, float* H, void* stream) {
+  if (!X || !H) return GPTQ_ERR_INVALID_ARG;
+  if (tokens < 0 || n_in <= 0) return GPTQ_ERR_INVALID_ARG;
+  if (x_dtype == GPTQ_F32) return GPTQ_ERR_UNSUPPORTED;
+  if (x_dtype != GPTQ_F16 && x_dtype != GPTQ_BF16) return GPTQ_ERR_INVALID_ARG;
+  if (n_in % 8 != 0 || n_in > 65535) return GPTQ_ERR_UNSUPPORTED;
+  if (!aligned16(X) || !aligned16(H)) return GPTQ_ERR_UNSUPPORTED;
+  if (tokens == 0) return GPTQ_OK;
+  return launch_hessian(X, x_dtype, tokens, n_in, H, static_cast<cudaStream_t>(stream));
+}
+
+int gptq_device_status(void* stream, int clear) {
+  return hessian_device_status(static_cast<cudaStream_t>(stream), clear);
+}
+
+int gptq_factor_hessian(const float* H, int64_t n_in, float damp_percent, int desc_act, float* U, int32_t* perm,
+                        void* stream) {
+  if (!H || !U || !perm) return GPTQ_ERR_INVALID_ARG;
+  if (n_in <= 0 || !valid_damp(damp_percent)) return GPTQ_ERR_INVALID_ARG;
+  if (n_in % 8 != 0 || n_in > 65535) return GPTQ_ERR_UNSUPPORTED;
+  if (!aligned16(H) || !aligned16(U) || !aligned16(perm)) return GPTQ_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t n = static_cast<size_t>(n_in);
+  Workspace ws;
+  GPTQ_TRY(alloc(ws, padded(n * n * 4) + padded(factor_small_bytes(n_in)) + padded(n * 4) + 512, s));
+  float* work = ws.take<float>(n * n);
+  void* small = ws.take<char>(factor_small_bytes(n_in));
+  int32_t* invperm = ws.take<int32_t>(n);
+  int* status = ws.take<int>(1);
+  GPTQ_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
+  GPTQ_TRY(factor_hessian(H, n_in, damp_percent, desc_act != 0, U, perm, invperm, work, small, status, s));
+  if (!desc_act) {
+    iota_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(perm, n_in);
+    GPTQ_TRY(after_launch());
+  }
+  return finish(status, s);
+}
+
+int gptq_quantize_layer_factored(const void* W, int w_dtype, int64_t n_out, int64_t n_in, const float* U,
+                                 const int32_t* perm, int bits, int group_size, int sym, int static_groups,
+                                 int blocksize, int32_t* qweight, float* scales, int32_t* zeros, int32_t* g_idx,
+                                 void* stream, gptq_stats* stats) {
+  GPTQ_TRY(check_quant_args(W, w_dtype, n_out, n_in, bits, group_size, blocksize, qweight, scales, zeros, g_idx));
+  if (!U || !perm) return GPTQ_ERR_INVALID_ARG;
+  if (!aligned16(U) || !aligned16(perm)) return GPTQ_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t no = static_cast<size_t>(n_out), ni = static_cast<size_t>(n_in);
+  Events evs;
+  GPTQ_TRY(evs.create(stats != nullptr));
+  Workspace ws;
+  GPTQ_TRY(alloc(ws, padded(no * ni * 4) + padded(no * ni) + padded(ni * 4) + 1024, s));
+  float* Wk = ws.take<float>(no * ni);
+  uint8_t* codesT = ws.take<uint8_t>(no * ni);
+  int32_t* invperm = ws.take<int32_t>(ni);
+  double* loss = ws.take<double>(1);
+  int* status = ws.take<int>(1);
+  GPTQ_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
+  const unsigned g1 = static_cast<unsigned>((ni + 255) / 256);
+  invert_perm_kernel<<<g1, 256, 0, s>>>(perm, n_in, invperm, status);
+  GPTQ_TRY(after_launch());
+  check_perm_kernel<<<g1, 256, 0, s>>>(perm, invperm, n_in, status);
+  GPTQ_TRY(after_launch());
+  GPTQ_TRY(sweep_common(W, w_dtype, n_out, n_in, U, perm, invperm, bits, group_size, sym, static_groups, blocksize,
+                        qweight, scales, zeros, g_idx, Wk, codesT, loss, status, s, stats, evs, 0));
+  if (stats) GPTQ_CUDA(cudaMemcpyAsync(&stats->damped_loss, loss, sizeof(double), cudaMemcpyDeviceToHost, s));
+  const int st = finish(status, s);
+  if (stats) {
+    stats->ms_prepare = evs.ms(0, 1);
+    stats->ms_factor = 0.f;
+    stats->ms_sweep = evs.ms(1, 2);
+    stats->ms_pack = evs.ms(2, 3);
+  }
+  return st;
+}
+
+int gptq_quantize_layer(const void* W, int w_dtype, int64_t n_out, int64_t n_in, const float* H, int bits,
+                        int group_size, float damp_percent, int sym, int desc_act, int static_groups, int blocksize,
+                        int32_t* qweight, float* scales, int32_t* zeros, int32_t* g_idx, void* stream,
+                        gptq_stats* stats) {
+  GPTQ_TRY(check_quant_args(W, w_dtype, n_out, n_in, bits, group_size, blocksize, qweight, scales, zeros, g_idx));
+  if (!H) return GPTQ_ERR_INVALID_ARG;
+  if (!valid_damp(damp_percent)) return GPTQ_ERR_INVALID_ARG;
+  if (!aligned16(H)) return GPTQ_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t no = static_cast<size_t>(n_out), ni = static_cast<size_t>(n_in);
+  Events evs;
+  GPTQ_TRY(evs.create(stats != nullptr));
+  Workspace ws;
+  GPTQ_TRY(alloc(ws,
+                 2 * padded(ni * ni * 4) + padded(factor_small_bytes(n_in)) + 2 * padded(ni * 4) +
+                     padded(no * ni * 4) + padded(no * ni) + 1024,
+                 s));
+  float* work = ws.take<float>(ni * ni);
+  float* U = ws.take<float>(ni * ni);
+  void* small = ws.take<char>(factor_small_bytes(n_in));
+  int32_t* perm = ws.take<int32_t>(ni);
+  int32_t* invperm = ws.take<int32_t>(ni);
+  float* Wk = ws.take<float>(no * ni);
+  uint8_t* codesT = ws.take<uint8_t>(no * ni);
+  double* loss = ws.take<double>(1);
+  int* status = ws.take<int>(1);
+  GPTQ_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
+  if (evs.on) GPTQ_CUDA(cudaEventRecord(evs.ev[4], s));
+  GPTQ_TRY(factor_hessian(H, n_in, damp_percent, desc_act != 0, U, perm, invperm, work, small, status, s));
+  if (evs.on) GPTQ_CUDA(cudaEventRecord(evs.ev[5], s));
+  GPTQ_TRY(sweep_common(W, w_dtype, n_out, n_in, U, desc_act ? perm : nullptr, desc_act ? invperm : nullptr, bits,
+                        group_size, sym, static_groups, blocksize, qweight, scales, zeros, g_idx, Wk, codesT, loss,
+                        status, s, stats, evs, 0));
+  if (stats) GPTQ_CUDA(cudaMemcpyAsync(&stats->damped_loss, loss, sizeof(double), cudaMemcpyDeviceToHost, s));
+  const int st = finish(status, s);
+  if (stats) {
+    stats->ms_factor = evs.ms(4, 5);
+    stats->ms_prepare = evs.ms(0, 1);
+    stats->ms_sweep = evs.ms(1, 2);
+    stats->ms_pack = evs.ms(2, 3);
+  }
+  return st;
+}
+
+}  // extern "C"

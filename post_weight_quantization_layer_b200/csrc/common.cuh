@@ -1,0 +1,102 @@
+// Shared host/device helpers of the GPTQ library (internal).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "../../include/gptq.h"
+
+namespace gptq {
+
+// Count of kernels launched by this library (reported by gptq_launch_count).
+extern std::atomic<uint64_t> g_launches;
+
+// Launch bookkeeping: count the launch and turn a launch error into a status.
+inline int after_launch() {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
+}
+
+#define GPTQ_TRY(expr)              \
+  do {                              \
+    int _st = (expr);               \
+    if (_st != GPTQ_OK) return _st; \
+  } while (0)
+
+#define GPTQ_CUDA(expr)                                 \
+  do {                                                  \
+    if ((expr) != cudaSuccess) { return GPTQ_ERR_CUDA; } \
+  } while (0)
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int num_sms() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms > 0 ? sms : 148;
+}
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T v);
+template <>
+__device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float to_f32<__half>(__half v) { return __half2float(v); }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// Device status word values shared by the kernels (same numbers as gptq_status).
+constexpr int kStatusNotPD = GPTQ_ERR_NOT_PD;
+constexpr int kStatusTimeout = GPTQ_ERR_TIMEOUT;
+
+// ---------------------------------------------------------------------------------------------
+// Internal entry points implemented in the other translation units.
+// All are stream-ordered; they return a gptq_status for host-side launch errors.
+
+// hessian.cu
+int launch_hessian(const void* X, int x_dtype, int64_t tokens, int64_t n, float* H, cudaStream_t s);
+int hessian_device_status(cudaStream_t s, int clear);
+
+// gemm_f32.cu: C[m,n] = beta*C[m,n] + alpha * sum_k A[m*lda+k] * B(k,n),
+// B(k,n) = transB ? B[n*ldb+k] : B[k*ldb+n].  upper != 0 skips 128x128 tiles of C
+// lying entirely below its diagonal (m > n for every element).
+int sgemm(cudaStream_t s, int64_t M, int64_t N, int64_t K, float alpha, const float* A, int64_t lda,
+          const float* B, int64_t ldb, bool transB, float beta, float* C, int64_t ldc, bool upper);
+
+// factor.cu: U (sweep order) and perm from H.  `work` holds n*n floats, `small` at least
+// factor_small_bytes(n) bytes; `status` is a device int.
+size_t factor_small_bytes(int64_t n);
+int factor_hessian(const float* H, int64_t n, float damp, bool desc_act, float* U, int32_t* perm,
+                   int32_t* invperm, float* work, void* small, int* status, cudaStream_t s);
+
+// sweep.cu: everything after the factor.
+struct SweepArgs {
+  const void* W;
+  int w_dtype;
+  int64_t n_out, n_in;
+  const float* U;
+  const int32_t* perm;     // nullptr = identity
+  const int32_t* invperm;  // nullptr = identity
+  int bits, group_size;
+  bool sym, static_groups;
+  int blocksize;
+  int32_t* qweight;
+  float* scales;
+  int32_t* zeros;
+  int32_t* g_idx;
+  // workspace
+  float* Wk;        // [n_out, n_in] fp32 working copy in sweep order
+  uint8_t* codesT;  // [n_in, n_out] codes in sweep order
+  double* loss;     // one double
+  int* status;
+  gptq_stats* stats;      // may be null
+  cudaEvent_t ev[4];      // valid when stats != null
+};
+int run_sweep(SweepArgs& a, cudaStream_t s, int* panel_width, int* outer_width);
+
+}  // namespace gptq

@@ -1,0 +1,439 @@
+// Quantize-and-compensate column sweep, lazy block updates, code packing.
+//
+// Source: "第5章 GPTQ 实战" §5.1.8 (the near-implementation pseudo-code): for each column
+// q, quantize with the group's fixed scale, form the normalised error
+// err = (w - q_int) / U[q, q], subtract err * U[q, later columns] from the columns of the
+// block not yet quantized, and after each block apply all of the block's errors to the
+// later columns at once as a matrix product (lazy batch update, key point 3).
+// §5.1.10: each group of group_size weights of a row shares one scale and zero point.
+// AutoGPTQ examples guide §1.4: sym / desc_act / static_groups.
+//
+// Work layout:
+// * Wk [n_out, n_in] fp32 is the working copy of W in sweep order.  Once column j is
+//   quantized its slot holds err_j, so the lazy updates read the errors in place.
+// * codesT [n_in, n_out] uint8 holds the codes in sweep order (column-major w.r.t. W),
+//   so both the sweep's writes and the packer's reads are coalesced across rows.
+// * Panels of P <= 128 columns: one kernel per panel, rows in parallel (8 threads per
+//   row, 16 columns per thread in registers, the panel's block of U in shared memory,
+//   group min/max and the error broadcast via warp shuffles).
+// * Two-level lazy updates: after each panel its errors update the rest of the current
+//   outer block (<= 1024 columns, L2-resident); after each outer block its errors update
+//   every later column in one GEMM with K = outer block width.
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace gptq {
+namespace {
+
+constexpr int PW = 128;                // max panel width
+constexpr int TPR = 8;                 // threads per row
+constexpr int NCOL = PW / TPR;         // columns per thread
+constexpr int ROWS = 256 / TPR;        // rows per CTA
+constexpr int PANEL_SMEM = PW * PW * 4 + PW * ROWS;
+
+// ---------------------------------------------------------------- quantizer (float32 decisions)
+__device__ __forceinline__ void params_sym(float amax, int bits, float& s, int& z) {
+  const int maxq = (1 << bits) - 1;
+  const float a = (amax == 0.f) ? 1.f : amax;
+  s = __fdiv_rn(__fmul_rn(2.f, a), static_cast<float>(maxq));
+  z = 1 << (bits - 1);
+}
+
+__device__ __forceinline__ void params_asym(float mn, float mx, int bits, float& s, int& z) {
+  const int maxq = (1 << bits) - 1;
+  float lo = fminf(0.f, mn), hi = fmaxf(0.f, mx);
+  if (hi == lo) {
+    lo = -1.f;
+    hi = 1.f;
+  }
+  s = __fdiv_rn(__fsub_rn(hi, lo), static_cast<float>(maxq));
+  const float zf = rintf(__fdiv_rn(-lo, s));
+  z = static_cast<int>(fminf(fmaxf(zf, 0.f), static_cast<float>(maxq)));
+}
+
+__device__ __forceinline__ void group_params(float mn, float mx, int bits, bool sym, float& s, int& z) {
+  if (sym)
+    params_sym(fmaxf(fabsf(mn), fabsf(mx)), bits, s, z);
+  else
+    params_asym(mn, mx, bits, s, z);
+}
+
+__device__ __forceinline__ int quant_code(float w, float s, int z, int maxq) {
+  const float r = rintf(__fdiv_rn(w, s));
+  const float q = fminf(fmaxf(__fadd_rn(r, static_cast<float>(z)), 0.f), static_cast<float>(maxq));
+  return static_cast<int>(q);
+}
+
+__device__ __forceinline__ int64_t clamp_idx(int32_t v, int64_t n) {
+  return v < 0 ? 0 : (v >= n ? n - 1 : v);
+}
+
+// ---------------------------------------------------------------- staging kernels
+template <typename T>
+__global__ void stage_weights_kernel(const T* __restrict__ W, int64_t n_out, int64_t n_in,
+                                     const int32_t* __restrict__ perm, float* __restrict__ Wk) {
+  const int64_t o = blockIdx.y;
+  for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < n_in;
+       j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t c = perm ? clamp_idx(perm[j], n_in) : j;
+    Wk[o * n_in + j] = to_f32(W[o * n_in + c]);
+  }
+}
+
+// Parameters fixed before the sweep: group_size == -1 (whole original row) or static
+// groups (consecutive original columns).  One warp per (group, row).
+template <typename T>
+__global__ void fixed_params_kernel(const T* __restrict__ W, int64_t n_out, int64_t n_in, int gsz, int64_t G,
+                                    int bits, int sym, float* __restrict__ scales, int32_t* __restrict__ zeros) {
+  const int64_t wid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid >= G * n_out) return;
+  const int64_t g = wid / n_out, o = wid % n_out;
+  const int64_t c0 = gsz < 0 ? 0 : g * gsz;
+  const int64_t c1 = gsz < 0 ? n_in : c0 + gsz;
+  float mn = INFINITY, mx = -INFINITY;
+  for (int64_t c = c0 + lane; c < c1; c += 32) {
+    const float v = to_f32(W[o * n_in + c]);
+    mn = fminf(mn, v);
+    mx = fmaxf(mx, v);
+  }
+  for (int off = 16; off; off >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  }
+  if (lane == 0) {
+    float s;
+    int z;
+    group_params(mn, mx, bits, sym != 0, s, z);
+    scales[g * n_out + o] = s;
+    zeros[g * n_out + o] = z;
+  }
+}
+
+// Non-static groups wider than a panel: parameters from the current (error-updated)
+// weights of sweep columns [j0, j0 + gsz) when the sweep reaches j0.  One warp per row.
+__global__ void current_params_kernel(const float* __restrict__ Wk, int64_t n_out, int64_t n_in, int64_t j0,
+                                      int gsz, int bits, int sym, float* __restrict__ scales,
+                                      int32_t* __restrict__ zeros) {
+  const int64_t o = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (o >= n_out) return;
+  float mn = INFINITY, mx = -INFINITY;
+  for (int64_t c = j0 + lane; c < j0 + gsz; c += 32) {
+    const float v = Wk[o * n_in + c];
+    mn = fminf(mn, v);
+    mx = fmaxf(mx, v);
+  }
+  for (int off = 16; off; off >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  }
+  if (lane == 0) {
+    float s;
+    int z;
+    group_params(mn, mx, bits, sym != 0, s, z);
+    scales[(j0 / gsz) * n_out + o] = s;
+    zeros[(j0 / gsz) * n_out + o] = z;
+  }
+}
+
+// ---------------------------------------------------------------- panel kernel
+struct PanelArgs {
+  float* Wk;
+  int64_t n_out, n_in;
+  const float* U;
+  int64_t j0;
+  int pw;
+  int bits, gsz;
+  int sym;
+  int in_panel_params;  // 1: non-static groups that start inside this panel
+  int static_groups;
+  const int32_t* perm;
+  float* scales;
+  int32_t* zeros;
+  uint8_t* codesT;
+  double* loss;
+};
+
+__global__ void __launch_bounds__(256) sweep_panel_kernel(PanelArgs a) {
+  extern __shared__ __align__(16) unsigned char psm[];
+  float* Us = reinterpret_cast<float*>(psm);               // [PW][PW], U[j0 + r][j0 + c]
+  uint8_t* cs = reinterpret_cast<uint8_t*>(Us + PW * PW);  // [PW][ROWS] codes of this CTA
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int tsub = tid % TPR;
+  const int rloc = tid / TPR;
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * ROWS;
+  const int64_t row = row0 + rloc;
+  const bool active = row < a.n_out;
+  const int pw = a.pw;
+  const int64_t j0 = a.j0, n_in = a.n_in, n_out = a.n_out;
+  const int maxq = (1 << a.bits) - 1;
+  const unsigned FULL = 0xffffffffu;
+  const int base_lane = lane & ~(TPR - 1);
+
+  for (int e = tid; e < PW * PW; e += 256) {
+    const int r = e / PW, c = e % PW;
+    Us[e] = (r < pw && c < pw && c >= r) ? a.U[(j0 + r) * n_in + j0 + c] : 0.f;
+  }
+  float v[NCOL];
+#pragma unroll
+  for (int m = 0; m < NCOL; ++m) {
+    const int col = tsub + TPR * m;
+    v[m] = (active && col < pw) ? a.Wk[row * n_in + j0 + col] : 0.f;
+  }
+  __syncthreads();
+
+  float s = 1.f;
+  int z = 0;
+  int64_t cur_g = -1;
+  double lsum = 0.0;
+
+#pragma unroll
+  for (int c = 0; c < PW; ++c) {
+    if (c < pw) {
+      const int64_t j = j0 + c;
+      if (a.in_panel_params) {
+        if (j % a.gsz == 0) {
+          float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+          for (int m = c / TPR; m < NCOL; ++m) {
+            const int col = tsub + TPR * m;
+            if (col >= c && col < c + a.gsz) {
+              mn = fminf(mn, v[m]);
+              mx = fmaxf(mx, v[m]);
+            }
+          }
+#pragma unroll
+          for (int off = 1; off < TPR; off <<= 1) {
+            mn = fminf(mn, __shfl_xor_sync(FULL, mn, off));
+            mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, off));
+          }
+          group_params(mn, mx, a.bits, a.sym != 0, s, z);
+          if (tsub == 0 && active) {
+            a.scales[(j / a.gsz) * n_out + row] = s;
+            a.zeros[(j / a.gsz) * n_out + row] = z;
+          }
+        }
+      } else {
+        int64_t g = 0;
+        if (a.gsz > 0) g = (a.static_groups && a.perm) ? clamp_idx(a.perm[j], n_in) / a.gsz : j / a.gsz;
+        if (g != cur_g) {
+          cur_g = g;
+          if (active) {
+            s = a.scales[g * n_out + row];
+            z = a.zeros[g * n_out + row];
+          }
+        }
+      }
+      float err = 0.f;
+      if (tsub == (c % TPR)) {
+        const float w = v[c / TPR];
+        const int q = quant_code(w, s, z, maxq);
+        const float what = __fmul_rn(s, static_cast<float>(q - z));
+        err = __fdiv_rn(__fsub_rn(w, what), Us[c * PW + c]);
+        v[c / TPR] = err;
+        cs[c * ROWS + rloc] = static_cast<uint8_t>(q);
+        lsum += static_cast<double>(err) * err;
+      }
+      err = __shfl_sync(FULL, err, base_lane + (c % TPR));
+#pragma unroll
+      for (int m = c / TPR; m < NCOL; ++m) {
+        const int col = tsub + TPR * m;
+        if (col > c) v[m] = fmaf(-err, Us[c * PW + col], v[m]);
+      }
+    }
+  }
+
+  // errors back into the working copy (they feed the lazy updates)
+#pragma unroll
+  for (int m = 0; m < NCOL; ++m) {
+    const int col = tsub + TPR * m;
+    if (active && col < pw) a.Wk[row * n_in + j0 + col] = v[m];
+  }
+  __syncthreads();
+  // codes: one 32-byte row segment per column
+  for (int e = tid; e < pw * ROWS; e += 256) {
+    const int c = e / ROWS, r = e % ROWS;
+    if (row0 + r < n_out) a.codesT[(j0 + c) * n_out + row0 + r] = cs[c * ROWS + r];
+  }
+  if (!active) lsum = 0.0;
+  for (int off = 16; off; off >>= 1) lsum += __shfl_xor_sync(FULL, lsum, off);
+  __shared__ double red[8];
+  if (lane == 0) red[tid >> 5] = lsum;
+  __syncthreads();
+  if (tid == 0) {
+    double t = 0.0;
+    for (int i = 0; i < 8; ++i) t += red[i];
+    atomicAdd(a.loss, t);
+  }
+}
+
+// ---------------------------------------------------------------- packing
+// qweight[w][o]: LSB-first stream of `bits`-bit codes along the ORIGINAL column order.
+// Sweep position of original column c is invperm[c].  Four outputs per thread -> one
+// 128-bit store when n_out % 4 == 0.
+__global__ void pack_kernel(const uint8_t* __restrict__ codesT, const int32_t* __restrict__ invperm, int64_t n_out,
+                            int64_t n_in, int bits, int32_t* __restrict__ qweight) {
+  const int64_t nw = n_in * bits / 32;
+  const int64_t o4 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
+  const int64_t w = blockIdx.y;
+  if (w >= nw || o4 >= n_out) return;
+  const int64_t bit0 = w * 32;
+  const int64_t cfirst = bit0 / bits, clast = (bit0 + 31) / bits;
+  uint32_t acc[4] = {0u, 0u, 0u, 0u};
+  const bool vec = (n_out % 4 == 0);
+  for (int64_t c = cfirst; c <= clast && c < n_in; ++c) {
+    const int64_t j = invperm ? clamp_idx(invperm[c], n_in) : c;
+    const int shift = static_cast<int>(c * bits - bit0);
+    uint32_t cv[4];
+    if (vec) {
+      const uchar4 q = *reinterpret_cast<const uchar4*>(codesT + j * n_out + o4);
+      cv[0] = q.x;
+      cv[1] = q.y;
+      cv[2] = q.z;
+      cv[3] = q.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) cv[e] = (o4 + e < n_out) ? codesT[j * n_out + o4 + e] : 0u;
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t m = cv[e] & ((1u << bits) - 1u);
+      acc[e] |= shift >= 0 ? (shift < 32 ? (m << shift) : 0u) : (m >> (-shift));
+    }
+  }
+  if (vec) {
+    *reinterpret_cast<int4*>(qweight + w * n_out + o4) =
+        make_int4(static_cast<int>(acc[0]), static_cast<int>(acc[1]), static_cast<int>(acc[2]), static_cast<int>(acc[3]));
+  } else {
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (o4 + e < n_out) qweight[w * n_out + o4 + e] = static_cast<int32_t>(acc[e]);
+  }
+}
+
+// g_idx[c] = group of original column c.
+__global__ void gidx_kernel(const int32_t* __restrict__ invperm, int64_t n_in, int gsz, int static_groups,
+                            int32_t* __restrict__ g_idx) {
+  const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (c >= n_in) return;
+  int64_t g = 0;
+  if (gsz > 0) {
+    const int64_t j = (invperm && !static_groups) ? clamp_idx(invperm[c], n_in) : c;
+    g = j / gsz;
+  }
+  g_idx[c] = static_cast<int32_t>(g);
+}
+
+template <typename T>
+int stage_and_fixed(const SweepArgs& a, cudaStream_t s) {
+  const T* W = static_cast<const T*>(a.W);
+  dim3 grid(static_cast<unsigned>(std::min<int64_t>((a.n_in + 255) / 256, 64)), static_cast<unsigned>(a.n_out));
+  stage_weights_kernel<T><<<grid, 256, 0, s>>>(W, a.n_out, a.n_in, a.perm, a.Wk);
+  GPTQ_TRY(after_launch());
+  if (a.group_size < 0 || a.static_groups) {
+    const int64_t G = a.group_size < 0 ? 1 : a.n_in / a.group_size;
+    const int64_t warps = G * a.n_out;
+    fixed_params_kernel<T><<<static_cast<unsigned>((warps * 32 + 255) / 256), 256, 0, s>>>(
+        W, a.n_out, a.n_in, a.group_size, G, a.bits, a.sym ? 1 : 0, a.scales, a.zeros);
+    GPTQ_TRY(after_launch());
+  }
+  return GPTQ_OK;
+}
+
+}  // namespace
+
+int run_sweep(SweepArgs& a, cudaStream_t s, int* panel_width, int* outer_width) {
+  static cudaError_t attr =
+      cudaFuncSetAttribute(sweep_panel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PANEL_SMEM);
+  if (attr != cudaSuccess) return GPTQ_ERR_CUDA;
+  const int64_t n_out = a.n_out, n_in = a.n_in;
+  const int g = a.group_size;
+  const bool dynamic_groups = g > 0 && !a.static_groups;
+
+  // Panel width: <= 128 and aligned to the groups whose parameters come from the
+  // current weights, so that a group's first column always sees every earlier error.
+  int P = PW;
+  if (dynamic_groups) {
+    if (g <= PW) {
+      P = (PW / g) * g;
+    } else {
+      P = 1;
+      for (int d = PW; d >= 1; --d)
+        if (g % d == 0) {
+          P = d;
+          break;
+        }
+    }
+  }
+  // Outer block: a multiple of P (and of g when groups are wider than a panel).
+  int64_t base = (dynamic_groups && g > P) ? g : P;
+  int64_t Q = base * std::max<int64_t>(1, 1024 / base);
+  if (panel_width) *panel_width = P;
+  if (outer_width) *outer_width = static_cast<int>(std::min<int64_t>(Q, n_in));
+
+  if (a.stats) GPTQ_CUDA(cudaEventRecord(a.ev[0], s));
+  GPTQ_CUDA(cudaMemsetAsync(a.loss, 0, sizeof(double), s));
+  if (a.w_dtype == GPTQ_F32)
+    GPTQ_TRY(stage_and_fixed<float>(a, s));
+  else if (a.w_dtype == GPTQ_F16)
+    GPTQ_TRY(stage_and_fixed<__half>(a, s));
+  else
+    GPTQ_TRY(stage_and_fixed<__nv_bfloat16>(a, s));
+  if (a.stats) GPTQ_CUDA(cudaEventRecord(a.ev[1], s));
+
+  PanelArgs pa;
+  pa.Wk = a.Wk;
+  pa.n_out = n_out;
+  pa.n_in = n_in;
+  pa.U = a.U;
+  pa.bits = a.bits;
+  pa.gsz = g;
+  pa.sym = a.sym ? 1 : 0;
+  pa.static_groups = a.static_groups ? 1 : 0;
+  pa.perm = a.perm;
+  pa.scales = a.scales;
+  pa.zeros = a.zeros;
+  pa.codesT = a.codesT;
+  pa.loss = a.loss;
+  const unsigned panel_grid = static_cast<unsigned>((n_out + ROWS - 1) / ROWS);
+
+  for (int64_t O0 = 0; O0 < n_in; O0 += Q) {
+    const int64_t O1 = std::min(O0 + Q, n_in);
+    for (int64_t p0 = O0; p0 < O1; p0 += P) {
+      const int64_t p1 = std::min(p0 + P, O1);
+      if (dynamic_groups && g > P && p0 % g == 0) {
+        current_params_kernel<<<static_cast<unsigned>((n_out * 32 + 255) / 256), 256, 0, s>>>(
+            a.Wk, n_out, n_in, p0, g, a.bits, a.sym ? 1 : 0, a.scales, a.zeros);
+        GPTQ_TRY(after_launch());
+      }
+      pa.j0 = p0;
+      pa.pw = static_cast<int>(p1 - p0);
+      pa.in_panel_params = (dynamic_groups && g <= P) ? 1 : 0;
+      sweep_panel_kernel<<<panel_grid, 256, PANEL_SMEM, s>>>(pa);
+      GPTQ_TRY(after_launch());
+      if (p1 < O1)  // rest of the outer block: W[:, p1:O1] -= Err[:, p0:p1] U[p0:p1, p1:O1]
+        GPTQ_TRY(sgemm(s, n_out, O1 - p1, p1 - p0, -1.f, a.Wk + p0, n_in, a.U + p0 * n_in + p1, n_in, false, 1.f,
+                       a.Wk + p1, n_in, false));
+    }
+    if (O1 < n_in)  // every later column: W[:, O1:] -= Err[:, O0:O1] U[O0:O1, O1:]
+      GPTQ_TRY(sgemm(s, n_out, n_in - O1, O1 - O0, -1.f, a.Wk + O0, n_in, a.U + O0 * n_in + O1, n_in, false, 1.f,
+                     a.Wk + O1, n_in, false));
+  }
+  if (a.stats) GPTQ_CUDA(cudaEventRecord(a.ev[2], s));
+
+  {
+    const int64_t nw = n_in * a.bits / 32;
+    dim3 grid(static_cast<unsigned>(((n_out + 3) / 4 + 127) / 128), static_cast<unsigned>(nw));
+    pack_kernel<<<grid, 128, 0, s>>>(a.codesT, a.invperm, n_out, n_in, a.bits, a.qweight);
+    GPTQ_TRY(after_launch());
+    gidx_kernel<<<static_cast<unsigned>((n_in + 255) / 256), 256, 0, s>>>(a.invperm, n_in, g,
+                                                                           a.static_groups ? 1 : 0, a.g_idx);
+    GPTQ_TRY(after_launch());
+  }
+  if (a.stats) GPTQ_CUDA(cudaEventRecord(a.ev[3], s));
+  return GPTQ_OK;
+}
+
+}  // namespace gptq

@@ -1,0 +1,63 @@
+"""GPU parity of gptq_factor_hessian: damping, act-order permutation and the
+upper Cholesky factor of the inverse, against the oracle's literal route."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import post_weight_quantization_layer_b200 as gq
+from post_weight_quantization_layer_b200 import synth
+from tests.gpu_util import device
+
+pytestmark = pytest.mark.gpu
+
+
+def _h(n, T, seed, dtype=torch.float16):
+    X = synth.HeavyChannelActs(n, T, seed, 0.02, 30.0, dtype).full()
+    return torch.from_numpy(O.hessian(X.double().numpy())).float()
+
+
+@pytest.mark.parametrize("n,T", [(256, 512), (264, 2000), (1032, 4096)])
+@pytest.mark.parametrize("desc_act", [False, True])
+def test_factor_matches_oracle(n, T, desc_act):
+    H = _h(n, T, n + T)
+    U, perm = gq.factor_hessian(H.to(device()), 0.01, desc_act)
+    torch.cuda.synchronize()
+    Hd64 = H.double().numpy()
+    p_ref = O.act_order_perm(Hd64) if desc_act else np.arange(n)
+    assert np.array_equal(perm.cpu().numpy(), p_ref)
+    Hd = O.dampen(Hd64[np.ix_(p_ref, p_ref)], 0.01)
+    U_ref = O.inverse_cholesky_upper(Hd)
+    Ug = U.cpu().double().numpy()
+    assert np.all(np.tril(Ug, -1) == 0)
+    assert np.all(np.diag(Ug) > 0)
+    # row-relative error of the compensation coefficients
+    err = np.abs(Ug - U_ref).max(axis=1) / np.abs(U_ref).max(axis=1)
+    assert err.max() < 2e-3, err.max()
+    # U^T U H_d = I up to fp32 factorisation error
+    R = Ug.T @ Ug @ Hd - np.eye(n)
+    assert np.abs(R).max() < 5e-3
+
+
+def test_not_positive_definite_is_reported():
+    dev = device()
+    with pytest.raises(gq.GPTQError) as e:
+        gq.factor_hessian(torch.zeros(64, 64, device=dev), 0.01)
+    assert e.value.status == 3
+    H = -torch.eye(128, device=dev)
+    with pytest.raises(gq.GPTQError) as e:
+        gq.factor_hessian(H, 0.01)
+    assert e.value.status == 3
+    # the context stays usable after the error
+    U, _ = gq.factor_hessian(torch.eye(64, device=dev) * 2, 0.01)
+    torch.cuda.synchronize()
+    assert torch.allclose(torch.diag(U).cpu(), torch.full((64,), (1 / 2.02) ** 0.5), rtol=1e-6)
+
+
+def test_act_order_ties_are_stable():
+    dev = device()
+    d = torch.tensor([3.0, 5.0, 3.0, 7.0, 5.0, 1.0, 7.0, 2.0])
+    H = torch.diag(d)
+    _, perm = gq.factor_hessian(H.to(dev), 0.01, True)
+    assert perm.cpu().tolist() == sorted(range(8), key=lambda i: (-float(d[i]), i))

@@ -1,0 +1,127 @@
+"""GPU parity of gptq_quantize_layer and the factor/sweep split against the oracle.
+
+Both sides receive the same W and the same fp32 Hessian (computed by the oracle
+from seeded activations and rounded to fp32)."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import post_weight_quantization_layer_b200 as gq
+from post_weight_quantization_layer_b200 import synth
+from tests.gpu_util import assert_parity, compare_quant, device
+
+pytestmark = pytest.mark.gpu
+
+
+def _problem(n_out, n_in, T, seed, w_dtype=torch.float16, x_dtype=torch.float16, outliers=True):
+    if outliers:
+        W = synth.outlier_weight(n_out, n_in, seed, dtype=w_dtype)
+    else:
+        W = synth.gaussian_weight(n_out, n_in, seed, dtype=w_dtype)
+    X = synth.StudentTActs(n_in, T, seed + 1, dtype=x_dtype).full()
+    H = torch.from_numpy(O.hessian(X.double().numpy())).float()
+    return W, H
+
+
+def _run(W, H, bits, g, sym, desc_act, static, blocksize=128, damp=0.01):
+    dev = device()
+    res = gq.quantize_layer(W.to(dev), H.to(dev), bits, g, damp, sym, desc_act, static, blocksize, stats=True)
+    torch.cuda.synchronize()
+    Wn, Hn = W.double().numpy(), H.double().numpy()
+    ref = O.gptq_quantize(Wn, Hn, bits, g, damp, sym, desc_act, static)  # eager sweep defines the result
+    return res, ref, compare_quant(res, ref, Wn, Hn, bits, W.shape[1])
+
+
+def test_tiny_config():
+    cfg = synth.CONFIGS["tiny"]
+    W = synth.weight_for(cfg, cfg.layers[0])
+    X = synth.acts_for(cfg, 0).full()
+    H = torch.from_numpy(O.hessian(X.double().numpy())).float()
+    res, ref, m = _run(W, H, cfg.bits, cfg.group_size, cfg.sym, cfg.desc_act, cfg.static_groups, cfg.blocksize)
+    assert_parity(m, "tiny")
+    assert abs(res.stats["damped_loss"] - ref["damped_loss"]) <= 0.01 * ref["damped_loss"]
+
+
+GRID = [(b, g, s, d, st) for b in (2, 3, 4, 8) for g in (32, 128, -1) for s in (True, False)
+        for d, st in ((False, False), (True, False), (True, True))]
+
+
+@pytest.mark.parametrize("bits,g,sym,desc_act,static", GRID)
+def test_config_grid(bits, g, sym, desc_act, static):
+    W, H = _problem(96, 512, 2048, 100 + bits * 7 + (g % 97))
+    _, _, m = _run(W, H, bits, g, sym, desc_act, static)
+    assert_parity(m, (bits, g, sym, desc_act, static))
+
+
+@pytest.mark.parametrize("n_out,n_in,g,bits", [(1, 256, 32, 4), (7, 200, -1, 4), (130, 264, 8, 4),
+                                              (33, 512, 256, 3), (64, 384, 384, 2), (5, 96, 96, 8),
+                                              (40, 1160, 40, 4)])
+def test_edge_shapes(n_out, n_in, g, bits):
+    """n_out = 1 and not a multiple of 4 (scalar pack path), ragged panels, groups wider
+    than a panel, a single group spanning all inputs, a group width not dividing 128."""
+    W, H = _problem(n_out, n_in, 4 * n_in, n_out * 31 + n_in, w_dtype=torch.float32)
+    _, _, m = _run(W, H, bits, g, True, False, False)
+    assert_parity(m, (n_out, n_in, g, bits))
+
+
+@pytest.mark.parametrize("blocksize", [1, 32, 128, 1000])
+def test_blocksize_does_not_change_results(blocksize):
+    W, H = _problem(64, 256, 1024, 9)
+    dev = device()
+    a = gq.quantize_layer(W.to(dev), H.to(dev), 4, 32, 0.01, True, True, False, blocksize)
+    b = gq.quantize_layer(W.to(dev), H.to(dev), 4, 32, 0.01, True, True, False, 128)
+    assert torch.equal(a.qweight, b.qweight) and torch.equal(a.scales, b.scales)
+
+
+@pytest.mark.parametrize("w_dtype", [torch.float32, torch.float16, torch.bfloat16])
+def test_weight_dtypes(w_dtype):
+    W, H = _problem(48, 256, 1024, 21, w_dtype=w_dtype)
+    _, _, m = _run(W, H, 4, 64, False, False, False)
+    assert_parity(m, str(w_dtype))
+
+
+def test_factored_sweep_with_oracle_factor():
+    """Sweep alone: GPU sweep given the oracle's U and permutation."""
+    W, H = _problem(128, 512, 2048, 33)
+    Hn = H.double().numpy()
+    perm = O.act_order_perm(Hn)
+    U = O.inverse_cholesky_upper(O.dampen(Hn[np.ix_(perm, perm)], 0.01))
+    dev = device()
+    res = gq.quantize_layer_factored(W.to(dev), torch.from_numpy(U).float().to(dev),
+                                     torch.from_numpy(perm.astype(np.int32)).to(dev), 4, 64, True, False, 128)
+    torch.cuda.synchronize()
+    ref = O.gptq_quantize(W.double().numpy(), Hn, 4, 64, 0.01, True, True, False)
+    m = compare_quant(res, ref, W.double().numpy(), Hn, 4, 512)
+    assert_parity(m, "factored")
+
+
+def test_factor_once_sweep_many_equals_quantize_layer():
+    W1, H = _problem(64, 256, 1024, 44)
+    W2 = synth.outlier_weight(80, 256, 45)
+    dev = device()
+    U, perm = gq.factor_hessian(H.to(dev), 0.01, True)
+    for W in (W1, W2):
+        a = gq.quantize_layer_factored(W.to(dev), U, perm, 4, 32, True, False, 128)
+        b = gq.quantize_layer(W.to(dev), H.to(dev), 4, 32, 0.01, True, True, False, 128)
+        assert torch.equal(a.qweight, b.qweight)
+        assert torch.equal(a.g_idx, b.g_idx)
+
+
+def test_invalid_permutation_is_rejected():
+    dev = device()
+    W, H = _problem(16, 64, 256, 3)
+    U, _ = gq.factor_hessian(H.to(dev), 0.01, False)
+    bad = torch.zeros(64, dtype=torch.int32, device=dev)
+    with pytest.raises(gq.GPTQError) as e:
+        gq.quantize_layer_factored(W.to(dev), U, bad, 4, 32)
+    assert e.value.status == 1
+
+
+def test_not_pd_through_quantize_layer():
+    dev = device()
+    W = torch.randn(16, 64, device=dev)
+    with pytest.raises(gq.GPTQError) as e:
+        gq.quantize_layer(W, torch.zeros(64, 64, device=dev), 4, 32)
+    assert e.value.status == 3

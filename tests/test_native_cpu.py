@@ -1,0 +1,101 @@
+"""CPU-side checks of the C ABI: the library loads, exports every declared
+symbol, and rejects bad arguments on the host before touching the GPU.
+
+Only rejection paths are exercised here: a call whose arguments pass host
+validation would enqueue GPU work.  Pointer arguments are fake but non-null
+and 16-byte aligned, so only the argument under test decides the outcome.
+"""
+
+import ctypes
+import math
+
+import pytest
+
+from post_weight_quantization_layer_b200 import _native
+from post_weight_quantization_layer_b200.build import build
+from tests.conftest import read_golden
+
+INVALID, UNSUPPORTED = 1, 2
+FAKE = ctypes.c_void_p(0x10000)
+MISALIGNED = ctypes.c_void_p(0x10004)
+
+
+@pytest.fixture(scope="module")
+def L():
+    build()
+    return _native.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = _native.declared_symbols()
+    assert set(names) >= {"gptq_accumulate_hessian", "gptq_quantize_layer", "gptq_status_string"}
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings_and_version(L):
+    for st in range(7):
+        assert L.gptq_status_string(st)
+    assert L.gptq_status_string(99) == b"unknown status"
+    assert L.gptq_version() >= 100
+
+
+def _quant(L, bits=4, g=128, damp=0.01, bs=128, n_out=64, n_in=256, dtype=1, W=FAKE, H=FAKE, out=FAKE):
+    return L.gptq_quantize_layer(W, dtype, n_out, n_in, H, bits, g, damp, 1, 0, 0, bs, out, out, out, out,
+                                 None, None)
+
+
+def test_validation_table_through_c_abi(L):
+    for ln in read_golden("validation.txt"):
+        bits, g, damp, bs, n_in, expect = ln.split()
+        if expect != "reject":
+            continue
+        st = _quant(L, int(bits), int(g), float(damp), int(bs), 64, int(n_in))
+        assert st == INVALID, ln
+
+
+def test_other_rejections(L):
+    assert _quant(L, W=None) == INVALID
+    assert _quant(L, H=None) == INVALID
+    assert _quant(L, out=None) == INVALID
+    assert _quant(L, dtype=7) == INVALID
+    assert _quant(L, n_out=0) == INVALID
+    assert _quant(L, n_in=-8) == INVALID
+    assert _quant(L, damp=math.nan) == INVALID
+    assert _quant(L, n_in=260, g=-1) == UNSUPPORTED          # n_in % 8
+    assert _quant(L, bits=3, n_in=264, g=-1) == UNSUPPORTED  # n_in*bits % 32
+    assert _quant(L, W=MISALIGNED) == UNSUPPORTED
+    assert _quant(L, n_in=70000, g=-1) == UNSUPPORTED
+
+
+def test_hessian_rejections(L):
+    acc = L.gptq_accumulate_hessian
+    assert acc(None, 1, 16, 64, FAKE, None) == INVALID
+    assert acc(FAKE, 1, 16, 64, None, None) == INVALID
+    assert acc(FAKE, 1, -1, 64, FAKE, None) == INVALID
+    assert acc(FAKE, 1, 16, 0, FAKE, None) == INVALID
+    assert acc(FAKE, 0, 16, 64, FAKE, None) == UNSUPPORTED   # fp32 activations
+    assert acc(FAKE, 5, 16, 64, FAKE, None) == INVALID
+    assert acc(FAKE, 2, 16, 60, FAKE, None) == UNSUPPORTED   # n_in % 8
+    assert acc(MISALIGNED, 2, 16, 64, FAKE, None) == UNSUPPORTED
+    assert acc(FAKE, 2, 0, 64, FAKE, None) == 0              # zero tokens: no-op, no GPU touched
+
+
+def test_factor_rejections(L):
+    f = L.gptq_factor_hessian
+    assert f(None, 64, 0.01, 0, FAKE, FAKE, None) == INVALID
+    assert f(FAKE, 64, 0.0, 0, FAKE, FAKE, None) == INVALID
+    assert f(FAKE, 64, 1.0, 0, FAKE, FAKE, None) == INVALID
+    assert f(FAKE, 64, math.nan, 0, FAKE, FAKE, None) == INVALID
+    assert f(FAKE, 60, 0.01, 0, FAKE, FAKE, None) == UNSUPPORTED
+    q = L.gptq_quantize_layer_factored
+    assert q(FAKE, 1, 64, 256, None, FAKE, 4, 128, 1, 0, 128, FAKE, FAKE, FAKE, FAKE, None, None) == INVALID
+    assert q(FAKE, 1, 64, 256, FAKE, FAKE, 6, 128, 1, 0, 128, FAKE, FAKE, FAKE, FAKE, None, None) == INVALID
+
+
+def test_python_binding_fails_loudly_without_cuda_tensors():
+    import torch
+
+    import post_weight_quantization_layer_b200 as gq
+    with pytest.raises(ValueError):
+        gq.quantize_layer(torch.zeros(4, 8), torch.zeros(8, 8))
