@@ -110,8 +110,9 @@ int gptq_accumulate_hessian(const void* X, int x_dtype, int64_t tokens, int64_t 
  *   g_idx   [n_in] int32: group of each original input column.
  *   Dequantized weight: scales[g_idx[c], o] * (code[o, c] - zeros[g_idx[c], o]).
  * n_in*bits % 32 != 0 or n_in % 8 != 0 -> UNSUPPORTED.
- * Workspace (about 2*n_in^2*4 + n_out*n_in*5 bytes) is allocated stream-ordered
- * inside the call (OOM if that fails).  The call is blocking: it synchronises
+ * Workspace (about 2*n_in^2*8 + n_out*n_in*17 bytes) is taken stream-ordered from a
+ * library-owned pool that keeps it cached for later calls (OOM if that fails; see
+ * gptq_trim_workspace).  The call is blocking: it synchronises
  * `stream` once at the end and returns NOT_PD if a pivot failed.
  * stats may be NULL.
  */
@@ -127,15 +128,17 @@ int gptq_quantize_layer(const void* W, int w_dtype, int64_t n_out, int64_t n_in,
  * Source: chapter 5 §5.1.8, damping and "Cholesky(inverse(H))".
  *
  * H     [n_in, n_in] fp32 symmetric, read-only.
- * U     [n_in, n_in] fp32 output: upper-triangular factor, in sweep order, of
+ * U     [n_in, n_in] fp64 output: upper-triangular factor, in sweep order, of
  *       the inverse of the damped (and, with desc_act, permuted) Hessian:
  *       inverse(H_d) = U^T U, U_jj > 0.  The strictly lower triangle is zero.
+ *       The factorisation is carried out in fp64: the sweep over thousands of
+ *       columns amplifies fp32-level error in U into different codes.
  * perm  [n_in] int32 output: sweep position j processes original column perm[j]
  *       (identity without desc_act).
  * Blocking; returns NOT_PD on a failed pivot.  UNSUPPORTED if n_in % 8 != 0.
  */
 int gptq_factor_hessian(const float* H, int64_t n_in, float damp_percent, int desc_act,
-                        float* U, int32_t* perm, void* stream);
+                        double* U, int32_t* perm, void* stream);
 
 /*
  * The sweep half: quantize W given the factor U and permutation perm produced
@@ -144,10 +147,17 @@ int gptq_factor_hessian(const float* H, int64_t n_in, float damp_percent, int de
  * Blocking.
  */
 int gptq_quantize_layer_factored(const void* W, int w_dtype, int64_t n_out, int64_t n_in,
-                                 const float* U, const int32_t* perm, int bits, int group_size,
+                                 const double* U, const int32_t* perm, int bits, int group_size,
                                  int sym, int static_groups, int blocksize,
                                  int32_t* qweight, float* scales, int32_t* zeros,
                                  int32_t* g_idx, void* stream, gptq_stats* stats);
+
+/*
+ * Release the device memory that the library's workspace pool keeps cached between
+ * calls on the current device (workspace is allocated stream-ordered from a pool owned
+ * by the library and reused across calls).  Synchronises the device first.
+ */
+int gptq_trim_workspace(void);
 
 /*
  * Synchronise `stream` and return the library's asynchronous device status

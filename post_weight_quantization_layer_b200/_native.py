@@ -46,6 +46,7 @@ _SIGNATURES = {
                                              c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
                                              c_void_p, ctypes.POINTER(GptqStats)]),
     "gptq_device_status": (c_int, [c_void_p, c_int]),
+    "gptq_trim_workspace": (c_int, []),
     "gptq_status_string": (ctypes.c_char_p, [c_int]),
     "gptq_launch_count": (ctypes.c_uint64, []),
     "gptq_version": (c_int, []),

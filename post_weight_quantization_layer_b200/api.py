@@ -110,10 +110,10 @@ def quantize_layer(W, H, bits=4, group_size=128, damp_percent=0.01, sym=True, de
 
 
 def factor_hessian(H, damp_percent=0.01, desc_act=False, stream=None):
-    """Returns (U, perm): inverse(H_d) = U^T U in sweep order, perm = column order."""
+    """Returns (U, perm): inverse(H_d) = U^T U in sweep order (fp64), perm = column order."""
     _need_cuda(H)
     n = H.shape[0]
-    U = torch.empty(n, n, dtype=torch.float32, device=H.device)
+    U = torch.empty(n, n, dtype=torch.float64, device=H.device)
     perm = torch.empty(n, dtype=torch.int32, device=H.device)
     st = lib().gptq_factor_hessian(_ptr(H), n, float(damp_percent), int(bool(desc_act)), _ptr(U), _ptr(perm),
                                    _stream(stream))
@@ -124,6 +124,8 @@ def factor_hessian(H, damp_percent=0.01, desc_act=False, stream=None):
 def quantize_layer_factored(W, U, perm, bits=4, group_size=128, sym=True, static_groups=False, blocksize=128,
                             stats=False, out=None, stream=None) -> QuantResult:
     _need_cuda(W, U, perm)
+    if U.dtype != torch.float64 or perm.dtype != torch.int32:
+        raise ValueError("U must be float64 and perm int32")
     n_out, n_in = W.shape
     qw, sc, zr, gi = _outputs(n_out, n_in, bits, group_size, W.device, out)
     st_obj = GptqStats() if stats else None

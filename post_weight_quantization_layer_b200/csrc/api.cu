@@ -1,6 +1,8 @@
 // extern "C" entry points: argument validation, workspace, orchestration, status.
 #include <cmath>
 #include <cstring>
+#include <map>
+#include <mutex>
 
 #include "common.cuh"
 
@@ -11,6 +13,34 @@ std::atomic<uint64_t> g_launches{0};
 namespace {
 
 constexpr int kVersion = 100;  // 0.1.0
+
+// Library-owned stream-ordered memory pool, one per device.  Its release threshold is
+// unbounded, so workspace memory is kept between calls instead of being returned to the
+// driver at every synchronisation (re-mapping hundreds of MB per call costs milliseconds).
+// gptq_trim_workspace() hands the cached memory back.
+std::mutex g_pool_mu;
+std::map<int, cudaMemPool_t> g_pools;
+
+cudaMemPool_t workspace_pool() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  std::lock_guard<std::mutex> lk(g_pool_mu);
+  auto it = g_pools.find(dev);
+  if (it != g_pools.end()) return it->second;
+  cudaMemPoolProps props = {};
+  props.allocType = cudaMemAllocationTypePinned;
+  props.location.type = cudaMemLocationTypeDevice;
+  props.location.id = dev;
+  cudaMemPool_t pool = nullptr;
+  if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  uint64_t thr = UINT64_MAX;
+  cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &thr);
+  g_pools[dev] = pool;
+  return pool;
+}
 
 // Stream-ordered workspace: one allocation carved into aligned pieces.
 struct Workspace {
@@ -34,7 +64,9 @@ size_t padded(size_t bytes) { return (bytes + 255) & ~size_t(255); }
 int alloc(Workspace& ws, size_t bytes, cudaStream_t s) {
   ws.s = s;
   ws.cap = bytes;
-  cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&ws.base), bytes, s);
+  cudaMemPool_t pool = workspace_pool();
+  if (!pool) return GPTQ_ERR_CUDA;
+  cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&ws.base), bytes, pool, s);
   if (e != cudaSuccess) {
     cudaGetLastError();
     ws.base = nullptr;
@@ -117,10 +149,11 @@ struct Events {
   }
 };
 
-int sweep_common(const void* W, int w_dtype, int64_t n_out, int64_t n_in, const float* U, const int32_t* perm,
+int sweep_common(const void* W, int w_dtype, int64_t n_out, int64_t n_in, const double* U, const int32_t* perm,
                  const int32_t* invperm, int bits, int group_size, int sym, int static_groups, int blocksize,
-                 int32_t* qweight, float* scales, int32_t* zeros, int32_t* g_idx, float* Wk, uint8_t* codesT,
-                 double* loss, int* status, cudaStream_t s, gptq_stats* stats, Events& evs, int ev0) {
+                 int32_t* qweight, float* scales, int32_t* zeros, int32_t* g_idx, double* Wk, double* Err,
+                 uint8_t* codesT, double* loss, int* status, cudaStream_t s, gptq_stats* stats, Events& evs,
+                 int ev0) {
   SweepArgs a;
   a.W = W;
   a.w_dtype = w_dtype;
@@ -139,6 +172,7 @@ int sweep_common(const void* W, int w_dtype, int64_t n_out, int64_t n_in, const 
   a.zeros = zeros;
   a.g_idx = g_idx;
   a.Wk = Wk;
+  a.Err = Err;
   a.codesT = codesT;
   a.loss = loss;
   a.status = status;
@@ -178,21 +212,28 @@ const char* gptq_status_string(int status) {
 }
 
 int gptq_accumulate_hessian(const void* X, int x_dtype, int64_t tokens, int64_t n_in, float* H, void* stream) {
-  if (!X || !H) return GPTQ_ERR_INVALID_ARG;
   if (tokens < 0 || n_in <= 0) return GPTQ_ERR_INVALID_ARG;
+  if (!H || (!X && tokens > 0)) return GPTQ_ERR_INVALID_ARG;
   if (x_dtype == GPTQ_F32) return GPTQ_ERR_UNSUPPORTED;
   if (x_dtype != GPTQ_F16 && x_dtype != GPTQ_BF16) return GPTQ_ERR_INVALID_ARG;
   if (n_in % 8 != 0 || n_in > 65535) return GPTQ_ERR_UNSUPPORTED;
+  if (tokens == 0) return GPTQ_OK;  // nothing to add; X may be NULL
   if (!aligned16(X) || !aligned16(H)) return GPTQ_ERR_UNSUPPORTED;
-  if (tokens == 0) return GPTQ_OK;
   return launch_hessian(X, x_dtype, tokens, n_in, H, static_cast<cudaStream_t>(stream));
+}
+
+int gptq_trim_workspace(void) {
+  cudaMemPool_t pool = workspace_pool();
+  if (!pool) return GPTQ_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return GPTQ_ERR_CUDA;
+  return cudaMemPoolTrimTo(pool, 0) == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
 }
 
 int gptq_device_status(void* stream, int clear) {
   return hessian_device_status(static_cast<cudaStream_t>(stream), clear);
 }
 
-int gptq_factor_hessian(const float* H, int64_t n_in, float damp_percent, int desc_act, float* U, int32_t* perm,
+int gptq_factor_hessian(const float* H, int64_t n_in, float damp_percent, int desc_act, double* U, int32_t* perm,
                         void* stream) {
   if (!H || !U || !perm) return GPTQ_ERR_INVALID_ARG;
   if (n_in <= 0 || !valid_damp(damp_percent)) return GPTQ_ERR_INVALID_ARG;
@@ -201,8 +242,8 @@ int gptq_factor_hessian(const float* H, int64_t n_in, float damp_percent, int de
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t n = static_cast<size_t>(n_in);
   Workspace ws;
-  GPTQ_TRY(alloc(ws, padded(n * n * 4) + padded(factor_small_bytes(n_in)) + padded(n * 4) + 512, s));
-  float* work = ws.take<float>(n * n);
+  GPTQ_TRY(alloc(ws, padded(factor_work_bytes(n_in)) + padded(factor_small_bytes(n_in)) + padded(n * 4) + 512, s));
+  void* work = ws.take<char>(factor_work_bytes(n_in));
   void* small = ws.take<char>(factor_small_bytes(n_in));
   int32_t* invperm = ws.take<int32_t>(n);
   int* status = ws.take<int>(1);
@@ -215,7 +256,7 @@ int gptq_factor_hessian(const float* H, int64_t n_in, float damp_percent, int de
   return finish(status, s);
 }
 
-int gptq_quantize_layer_factored(const void* W, int w_dtype, int64_t n_out, int64_t n_in, const float* U,
+int gptq_quantize_layer_factored(const void* W, int w_dtype, int64_t n_out, int64_t n_in, const double* U,
                                  const int32_t* perm, int bits, int group_size, int sym, int static_groups,
                                  int blocksize, int32_t* qweight, float* scales, int32_t* zeros, int32_t* g_idx,
                                  void* stream, gptq_stats* stats) {
@@ -227,8 +268,9 @@ int gptq_quantize_layer_factored(const void* W, int w_dtype, int64_t n_out, int6
   Events evs;
   GPTQ_TRY(evs.create(stats != nullptr));
   Workspace ws;
-  GPTQ_TRY(alloc(ws, padded(no * ni * 4) + padded(no * ni) + padded(ni * 4) + 1024, s));
-  float* Wk = ws.take<float>(no * ni);
+  GPTQ_TRY(alloc(ws, 2 * padded(no * ni * 8) + padded(no * ni) + padded(ni * 4) + 1024, s));
+  double* Wk = ws.take<double>(no * ni);
+  double* Err = ws.take<double>(no * ni);
   uint8_t* codesT = ws.take<uint8_t>(no * ni);
   int32_t* invperm = ws.take<int32_t>(ni);
   double* loss = ws.take<double>(1);
@@ -240,7 +282,7 @@ int gptq_quantize_layer_factored(const void* W, int w_dtype, int64_t n_out, int6
   check_perm_kernel<<<g1, 256, 0, s>>>(perm, invperm, n_in, status);
   GPTQ_TRY(after_launch());
   GPTQ_TRY(sweep_common(W, w_dtype, n_out, n_in, U, perm, invperm, bits, group_size, sym, static_groups, blocksize,
-                        qweight, scales, zeros, g_idx, Wk, codesT, loss, status, s, stats, evs, 0));
+                        qweight, scales, zeros, g_idx, Wk, Err, codesT, loss, status, s, stats, evs, 0));
   if (stats) GPTQ_CUDA(cudaMemcpyAsync(&stats->damped_loss, loss, sizeof(double), cudaMemcpyDeviceToHost, s));
   const int st = finish(status, s);
   if (stats) {
@@ -266,15 +308,16 @@ int gptq_quantize_layer(const void* W, int w_dtype, int64_t n_out, int64_t n_in,
   GPTQ_TRY(evs.create(stats != nullptr));
   Workspace ws;
   GPTQ_TRY(alloc(ws,
-                 2 * padded(ni * ni * 4) + padded(factor_small_bytes(n_in)) + 2 * padded(ni * 4) +
-                     padded(no * ni * 4) + padded(no * ni) + 1024,
+                 padded(factor_work_bytes(n_in)) + padded(ni * ni * 8) + padded(factor_small_bytes(n_in)) +
+                     2 * padded(ni * 4) + 2 * padded(no * ni * 8) + padded(no * ni) + 1024,
                  s));
-  float* work = ws.take<float>(ni * ni);
-  float* U = ws.take<float>(ni * ni);
+  void* work = ws.take<char>(factor_work_bytes(n_in));
+  double* U = ws.take<double>(ni * ni);
   void* small = ws.take<char>(factor_small_bytes(n_in));
   int32_t* perm = ws.take<int32_t>(ni);
   int32_t* invperm = ws.take<int32_t>(ni);
-  float* Wk = ws.take<float>(no * ni);
+  double* Wk = ws.take<double>(no * ni);
+  double* Err = ws.take<double>(no * ni);
   uint8_t* codesT = ws.take<uint8_t>(no * ni);
   double* loss = ws.take<double>(1);
   int* status = ws.take<int>(1);
@@ -283,8 +326,8 @@ int gptq_quantize_layer(const void* W, int w_dtype, int64_t n_out, int64_t n_in,
   GPTQ_TRY(factor_hessian(H, n_in, damp_percent, desc_act != 0, U, perm, invperm, work, small, status, s));
   if (evs.on) GPTQ_CUDA(cudaEventRecord(evs.ev[5], s));
   GPTQ_TRY(sweep_common(W, w_dtype, n_out, n_in, U, desc_act ? perm : nullptr, desc_act ? invperm : nullptr, bits,
-                        group_size, sym, static_groups, blocksize, qweight, scales, zeros, g_idx, Wk, codesT, loss,
-                        status, s, stats, evs, 0));
+                        group_size, sym, static_groups, blocksize, qweight, scales, zeros, g_idx, Wk, Err, codesT,
+                        loss, status, s, stats, evs, 0));
   if (stats) GPTQ_CUDA(cudaMemcpyAsync(&stats->damped_loss, loss, sizeof(double), cudaMemcpyDeviceToHost, s));
   const int st = finish(status, s);
   if (stats) {

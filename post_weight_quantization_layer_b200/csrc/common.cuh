@@ -62,24 +62,32 @@ constexpr int kStatusTimeout = GPTQ_ERR_TIMEOUT;
 int launch_hessian(const void* X, int x_dtype, int64_t tokens, int64_t n, float* H, cudaStream_t s);
 int hessian_device_status(cudaStream_t s, int clear);
 
-// gemm_f32.cu: C[m,n] = beta*C[m,n] + alpha * sum_k A[m*lda+k] * B(k,n),
+// gemm.cu: C[m,n] = beta*C[m,n] + alpha * sum_k A[m*lda+k] * B(k,n),
 // B(k,n) = transB ? B[n*ldb+k] : B[k*ldb+n].  upper != 0 skips 128x128 tiles of C
 // lying entirely below its diagonal (m > n for every element).
 int sgemm(cudaStream_t s, int64_t M, int64_t N, int64_t K, float alpha, const float* A, int64_t lda,
           const float* B, int64_t ldb, bool transB, float beta, float* C, int64_t ldc, bool upper);
+// Same product (fp32 operands, fp32 accumulation) applied to an fp64 C:
+// C[m,n] = C[m,n] + (double)(alpha * sum_k A[m,k] B(k,n)).
+int sgemm_acc64(cudaStream_t s, int64_t M, int64_t N, int64_t K, float alpha, const float* A, int64_t lda,
+                const float* B, int64_t ldb, double* C, int64_t ldc);
+// fp64 operands, fp64 accumulation (same conventions as sgemm).
+int dgemm(cudaStream_t s, int64_t M, int64_t N, int64_t K, double alpha, const double* A, int64_t lda,
+          const double* B, int64_t ldb, bool transB, double beta, double* C, int64_t ldc, bool upper);
 
-// factor.cu: U (sweep order) and perm from H.  `work` holds n*n floats, `small` at least
-// factor_small_bytes(n) bytes; `status` is a device int.
+// factor.cu: U (sweep order, fp64) and perm from H.  `work` holds factor_work_bytes(n),
+// `small` factor_small_bytes(n); `status` is a device int.
 size_t factor_small_bytes(int64_t n);
-int factor_hessian(const float* H, int64_t n, float damp, bool desc_act, float* U, int32_t* perm,
-                   int32_t* invperm, float* work, void* small, int* status, cudaStream_t s);
+size_t factor_work_bytes(int64_t n);
+int factor_hessian(const float* H, int64_t n, float damp, bool desc_act, double* U, int32_t* perm,
+                   int32_t* invperm, void* work, void* small, int* status, cudaStream_t s);
 
 // sweep.cu: everything after the factor.
 struct SweepArgs {
   const void* W;
   int w_dtype;
   int64_t n_out, n_in;
-  const float* U;
+  const double* U;
   const int32_t* perm;     // nullptr = identity
   const int32_t* invperm;  // nullptr = identity
   int bits, group_size;
@@ -90,7 +98,8 @@ struct SweepArgs {
   int32_t* zeros;
   int32_t* g_idx;
   // workspace
-  float* Wk;        // [n_out, n_in] fp32 working copy in sweep order
+  double* Wk;       // [n_out, n_in] fp64 working copy of the weights, sweep order
+  double* Err;      // [n_out, n_in] fp64 normalised errors, sweep order
   uint8_t* codesT;  // [n_in, n_out] codes in sweep order
   double* loss;     // one double
   int* status;

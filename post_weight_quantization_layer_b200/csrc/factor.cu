@@ -11,9 +11,15 @@
 // damped Hessian from the bottom-right corner, H_d = V V^T with V upper triangular,
 // and invert V: inverse(H_d) = V^-T V^-1, so U = V^-1 is exactly the upper factor
 // with inverse(H_d) = U^T U and a positive diagonal (2n^3/3 flops).  Both steps are
-// blocked with 128-wide blocks: a single-CTA kernel factors and inverts each diagonal
+// blocked with 64-wide blocks: a single-CTA kernel factors and inverts each diagonal
 // block in shared memory (and checks every pivot), and the off-diagonal work runs as
 // GEMMs.
+//
+// Precision: the factorisation runs in fp64 and U stays fp64.  The forward error of a
+// Cholesky factor grows like cond(H_d) times the working precision; with cond(H_d) ~ 1e4
+// (heavy-tailed activation channels) an fp32 factorisation leaves ~1e-5 relative error
+// in U, and a sweep over thousands of columns amplifies even fp32 rounding of U into
+// different codes.
 #include <algorithm>
 
 #include "common.cuh"
@@ -21,9 +27,10 @@
 namespace gptq {
 namespace {
 
-constexpr int NB = 128;  // block width of the factorisation
+constexpr int NB = 64;  // block width of the factorisation
 constexpr int DIAG_THREADS = 512;
 constexpr int SP = NB + 1;  // padded pitch of the diagonal block in shared memory
+using real = double;     // working precision of the factorisation
 
 // Sum of diag(H) in double.
 __global__ void diag_sum_kernel(const float* __restrict__ H, int64_t n, double* out) {
@@ -68,14 +75,14 @@ __global__ void act_order_rank_kernel(const float* __restrict__ H, int64_t n, in
 
 // A = P H P^T + lambda I with lambda = damp * mean(diag H) (P = permutation, or none).
 __global__ void permute_damp_kernel(const float* __restrict__ H, int64_t n, const int32_t* __restrict__ perm,
-                                    const double* __restrict__ diag_sum, float damp, float* __restrict__ A) {
+                                    const double* __restrict__ diag_sum, float damp, real* __restrict__ A) {
   const int64_t i = blockIdx.y;
   const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (j >= n) return;
   const int64_t pi = perm ? perm[i] : i;
   const int64_t pj = perm ? perm[j] : j;
-  float v = H[pi * n + pj];
-  if (i == j) v += static_cast<float>(static_cast<double>(damp) * (*diag_sum / static_cast<double>(n)));
+  real v = H[pi * n + pj];
+  if (i == j) v += static_cast<double>(damp) * (*diag_sum / static_cast<double>(n));
   A[i * n + j] = v;
 }
 
@@ -83,55 +90,106 @@ __global__ void permute_damp_kernel(const float* __restrict__ H, int64_t n, cons
 // write V back into A, and its inverse into Winv[k0:k0+nb, 0:nb] (ld NB).  A pivot that is
 // not positive and finite sets *status = NOT_PD; the factorisation continues with a unit
 // pivot so that every later kernel still sees finite numbers.
-__global__ void __launch_bounds__(DIAG_THREADS) chol_diag_kernel(float* A, int64_t lda, int64_t k0, int nb,
-                                                                 float* Winv, int* status) {
-  extern __shared__ float sm[];
-  float* S = sm;              // V, [NB][SP]
-  float* X = sm + NB * SP;    // V^-1, [NB][SP]
-  float* col = X + NB * SP;   // scaled column, [NB]
+//
+// The block is padded to NB x NB with an identity in its bottom-right corner (no coupling),
+// which leaves the real part of V and V^-1 unchanged and lets every size use the same
+// power-of-two inverse below.
+__global__ void __launch_bounds__(DIAG_THREADS) chol_diag_kernel(real* A, int64_t lda, int64_t k0, int nb,
+                                                                 real* Winv, int* status) {
+  extern __shared__ real sm[];
+  real* S = sm;              // V, [NB][SP]
+  real* X = sm + NB * SP;    // V^-1, [NB][SP]
+  real* T = X + NB * SP;     // product scratch, [NB/2][SP]
+  real* col = T + (NB / 2) * SP;  // scaled column, [NB]
   __shared__ int bad;
   const int tid = threadIdx.x;
   if (tid == 0) bad = 0;
-  for (int e = tid; e < nb * nb; e += DIAG_THREADS) {
-    const int i = e / nb, j = e % nb;
-    S[i * SP + j] = (i <= j) ? A[(k0 + i) * lda + k0 + j] : 0.f;
+  for (int e = tid; e < NB * NB; e += DIAG_THREADS) {
+    const int i = e / NB, j = e % NB;
+    real v = 0;
+    if (i < nb && j < nb) {
+      if (i <= j) v = A[(k0 + i) * lda + k0 + j];
+    } else if (i == j) {
+      v = 1;
+    }
+    S[i * SP + j] = v;
+    X[i * SP + j] = 0;
+  }
+  // Each thread owns fixed elements (i <= j) of the upper triangle for the rank-1 updates.
+  constexpr int NUP = NB * (NB + 1) / 2;
+  constexpr int SLOTS = (NUP + DIAG_THREADS - 1) / DIAG_THREADS;
+  int own[SLOTS];
+#pragma unroll
+  for (int r = 0; r < SLOTS; ++r) {
+    int e = tid + r * DIAG_THREADS, i = 0;
+    if (e < NUP) {
+      while (e >= NB - i) {
+        e -= NB - i;
+        ++i;
+      }
+      own[r] = (i << 8) | (i + e);
+    } else {
+      own[r] = -1;
+    }
   }
   __syncthreads();
-  for (int c = nb - 1; c >= 0; --c) {
-    float d = S[c * SP + c];
-    if (!(d > 0.f) || !isfinite(d)) {
+  for (int c = NB - 1; c >= 0; --c) {
+    real d = S[c * SP + c];
+    if (!(d > 0) || !isfinite(d)) {
       if (tid == 0) bad = 1;
-      d = 1.f;
+      d = 1;
     }
-    const float v = sqrtf(d);
+    const real v = sqrt(d);
     if (tid < c) col[tid] = S[tid * SP + c] / v;
     __syncthreads();
     if (tid == 0) S[c * SP + c] = v;
     if (tid < c) S[tid * SP + c] = col[tid];
-    const int cc = c * c;
-    for (int e = tid; e < cc; e += DIAG_THREADS) {
-      const int i = e / c, j = e - i * c;
-      if (i <= j) S[i * SP + j] = fmaf(-col[i], col[j], S[i * SP + j]);
+#pragma unroll
+    for (int r = 0; r < SLOTS; ++r) {
+      const int o = own[r];
+      const int i = o >> 8, j = o & 255;
+      if (o >= 0 && j < c) S[i * SP + j] = fma(-col[i], col[j], S[i * SP + j]);
     }
     __syncthreads();
   }
-  // X = V^-1 (upper): thread j solves column j by back substitution.
-  if (tid < nb) {
-    const int j = tid;
-    X[j * SP + j] = 1.f / S[j * SP + j];
-    for (int i = j - 1; i >= 0; --i) {
-      float s0 = 0.f, s1 = 0.f;
-      int l = i + 1;
-      for (; l + 1 <= j; l += 2) {
-        s0 = fmaf(S[i * SP + l], X[l * SP + j], s0);
-        s1 = fmaf(S[i * SP + l + 1], X[(l + 1) * SP + j], s1);
+
+  // X = V^-1 by doubling: invert 16x16 diagonal blocks, then join neighbours with
+  // [[A, B], [0, C]]^-1 = [[A^-1, -A^-1 B C^-1], [0, C^-1]].
+  {
+    const int warp = tid >> 5, lane = tid & 31;
+    if (warp < NB / 16 && lane < 16) {
+      const int p = warp * 16, j = p + lane;
+      X[j * SP + j] = 1 / S[j * SP + j];
+      for (int i = j - 1; i >= p; --i) {
+        real acc = 0;
+        for (int l = i + 1; l <= j; ++l) acc = fma(S[i * SP + l], X[l * SP + j], acc);
+        X[i * SP + j] = -acc / S[i * SP + i];
       }
-      if (l <= j) s0 = fmaf(S[i * SP + l], X[l * SP + j], s0);
-      X[i * SP + j] = -(s0 + s1) / S[i * SP + i];
     }
-    for (int i = j + 1; i < nb; ++i) X[i * SP + j] = 0.f;
+    __syncthreads();
   }
-  __syncthreads();
+  for (int sz = 16; sz < NB; sz *= 2) {
+    const int pairs = NB / (2 * sz);
+    // T = B * C^-1 for every pair (B: rows p..p+sz, cols p+sz..p+2sz of V)
+    for (int e = tid; e < pairs * sz * sz; e += DIAG_THREADS) {
+      const int pr = e / (sz * sz), r = (e / sz) % sz, cc = e % sz;
+      const int p = pr * 2 * sz;
+      real acc = 0;
+      for (int l = 0; l <= cc; ++l) acc = fma(S[(p + r) * SP + p + sz + l], X[(p + sz + l) * SP + p + sz + cc], acc);
+      T[(pr * sz + r) * SP + cc] = acc;
+    }
+    __syncthreads();
+    // X12 = -A^-1 * T
+    for (int e = tid; e < pairs * sz * sz; e += DIAG_THREADS) {
+      const int pr = e / (sz * sz), r = (e / sz) % sz, cc = e % sz;
+      const int p = pr * 2 * sz;
+      real acc = 0;
+      for (int l = r; l < sz; ++l) acc = fma(X[(p + r) * SP + p + l], T[(pr * sz + l) * SP + cc], acc);
+      X[(p + r) * SP + p + sz + cc] = -acc;
+    }
+    __syncthreads();
+  }
+
   for (int e = tid; e < nb * nb; e += DIAG_THREADS) {
     const int i = e / nb, j = e % nb;
     if (i <= j) A[(k0 + i) * lda + k0 + j] = S[i * SP + j];
@@ -140,27 +198,30 @@ __global__ void __launch_bounds__(DIAG_THREADS) chol_diag_kernel(float* A, int64
   if (tid == 0 && bad) atomicExch(status, kStatusNotPD);
 }
 
-__global__ void set_diag_kernel(float* R, int64_t n, float v) {
+__global__ void set_diag_kernel(real* R, int64_t n, real v) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i < n) R[i * n + i] = v;
 }
 
-constexpr int DIAG_SMEM = (2 * NB * SP + NB) * static_cast<int>(sizeof(float));
+constexpr int DIAG_SMEM = (2 * NB * SP + (NB / 2) * SP + NB) * static_cast<int>(sizeof(real));
 
 }  // namespace
 
 size_t factor_small_bytes(int64_t n) {
-  return static_cast<size_t>(n) * NB * sizeof(float) + 256;
+  return static_cast<size_t>(n) * NB * sizeof(real) + 256;
 }
 
-int factor_hessian(const float* H, int64_t n, float damp, bool desc_act, float* U, int32_t* perm,
-                   int32_t* invperm, float* work, void* small, int* status, cudaStream_t s) {
+size_t factor_work_bytes(int64_t n) { return static_cast<size_t>(n) * n * sizeof(real); }
+
+int factor_hessian(const float* H, int64_t n, float damp, bool desc_act, double* U, int32_t* perm,
+                   int32_t* invperm, void* work, void* small, int* status, cudaStream_t s) {
   static cudaError_t attr = cudaFuncSetAttribute(chol_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  DIAG_SMEM);
   if (attr != cudaSuccess) return GPTQ_ERR_CUDA;
   double* dsum = reinterpret_cast<double*>(small);
-  float* Winv = reinterpret_cast<float*>(static_cast<char*>(small) + 256);
-  float* A = work;
+  real* Winv = reinterpret_cast<real*>(static_cast<char*>(small) + 256);
+  real* A = static_cast<real*>(work);   // damped Hessian, then V
+  real* R = U;                          // V^-1, written in place into the output
 
   GPTQ_CUDA(cudaMemsetAsync(dsum, 0, sizeof(double), s));
   diag_sum_kernel<<<std::min<int64_t>((n + 255) / 256, 148), 256, 0, s>>>(H, n, dsum);
@@ -169,11 +230,9 @@ int factor_hessian(const float* H, int64_t n, float damp, bool desc_act, float* 
     act_order_rank_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(H, n, perm, invperm);
     GPTQ_TRY(after_launch());
   }
-  {
-    dim3 grid(static_cast<unsigned>((n + 255) / 256), static_cast<unsigned>(n));
-    permute_damp_kernel<<<grid, 256, 0, s>>>(H, n, desc_act ? perm : nullptr, dsum, damp, A);
-    GPTQ_TRY(after_launch());
-  }
+  const dim3 rgrid(static_cast<unsigned>((n + 255) / 256), static_cast<unsigned>(n));
+  permute_damp_kernel<<<rgrid, 256, 0, s>>>(H, n, desc_act ? perm : nullptr, dsum, damp, A);
+  GPTQ_TRY(after_launch());
 
   // Reverse (bottom-right first) blocked Cholesky: A -> V (upper), H_d = V V^T.
   const int64_t nblk = (n + NB - 1) / NB;
@@ -184,25 +243,25 @@ int factor_hessian(const float* H, int64_t n, float damp, bool desc_act, float* 
     GPTQ_TRY(after_launch());
     if (k0 > 0) {
       // Panel: V[0:k0, k] = A[0:k0, k] * V_kk^-T   (in place; N = nb <= 128)
-      GPTQ_TRY(sgemm(s, k0, nb, nb, 1.f, A + k0, n, Winv + k0 * NB, NB, true, 0.f, A + k0, n, false));
+      GPTQ_TRY(dgemm(s, k0, nb, nb, 1.0, A + k0, n, Winv + k0 * NB, NB, true, 0.0, A + k0, n, false));
       // Trailing: A[0:k0, 0:k0] -= V[0:k0, k] V[0:k0, k]^T   (upper tiles only)
-      GPTQ_TRY(sgemm(s, k0, k0, nb, -1.f, A + k0, n, A + k0, n, true, 1.f, A, n, true));
+      GPTQ_TRY(dgemm(s, k0, k0, nb, -1.0, A + k0, n, A + k0, n, true, 1.0, A, n, true));
     }
   }
 
-  // U = V^-1 by block back substitution on the identity, bottom block row first.
-  GPTQ_CUDA(cudaMemsetAsync(U, 0, static_cast<size_t>(n) * n * sizeof(float), s));
-  set_diag_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(U, n, 1.f);
+  // R = V^-1 by block back substitution on the identity, bottom block row first.
+  GPTQ_CUDA(cudaMemsetAsync(R, 0, static_cast<size_t>(n) * n * sizeof(real), s));
+  set_diag_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(R, n, 1.0);
   GPTQ_TRY(after_launch());
   for (int64_t k = nblk - 1; k >= 0; --k) {
     const int64_t k0 = k * NB;
     const int nb = static_cast<int>(std::min<int64_t>(NB, n - k0));
-    // U[k, k0:] = V_kk^-1 * R[k, k0:]   (in place; M = nb <= 128)
-    GPTQ_TRY(sgemm(s, nb, n - k0, nb, 1.f, Winv + k0 * NB, NB, U + k0 * n + k0, n, false, 0.f, U + k0 * n + k0, n,
+    // R[k, k0:] = V_kk^-1 * R[k, k0:]   (in place; M = nb <= 128)
+    GPTQ_TRY(dgemm(s, nb, n - k0, nb, 1.0, Winv + k0 * NB, NB, R + k0 * n + k0, n, false, 0.0, R + k0 * n + k0, n,
                    false));
     if (k0 > 0) {
-      // R[0:k0, k0:] -= V[0:k0, k] * U[k, k0:]
-      GPTQ_TRY(sgemm(s, k0, n - k0, nb, -1.f, A + k0, n, U + k0 * n + k0, n, false, 1.f, U + k0, n, false));
+      // R[0:k0, k0:] -= V[0:k0, k] * R[k, k0:]
+      GPTQ_TRY(dgemm(s, k0, n - k0, nb, -1.0, A + k0, n, R + k0 * n + k0, n, false, 1.0, R + k0, n, false));
     }
   }
   return GPTQ_OK;

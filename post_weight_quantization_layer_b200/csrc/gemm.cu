@@ -1,5 +1,5 @@
-// FP32 GEMM on the CUDA cores, used for the rank-k updates of the factorisation and the
-// lazy block updates of the sweep: C = beta*C + alpha * A * op(B).
+// GEMM on the CUDA cores in fp32 (lazy block updates of the sweep) and fp64 (rank-k
+// updates of the factorisation): C = beta*C + alpha * A * op(B).
 //
 // 128x128 tile per 256-thread CTA, 8x8 outputs per thread, K staged 8 at a time through
 // double-buffered shared memory.  All operands are row-major with arbitrary leading
@@ -15,36 +15,35 @@ namespace {
 
 constexpr int TM = 128, TN = 128, TK = 8, PAD = 4;
 
-template <bool TRANSB>
-__global__ void __launch_bounds__(256) sgemm_kernel(int64_t M, int64_t N, int64_t K, float alpha,
-                                                    const float* A, int64_t lda,
-                                                    const float* B, int64_t ldb, float beta,
-                                                    float* C, int64_t ldc, int upper) {
+template <typename T, bool TRANSB, typename CT>
+__global__ void __launch_bounds__(256) gemm_kernel(int64_t M, int64_t N, int64_t K, T alpha, const T* A,
+                                                   int64_t lda, const T* B, int64_t ldb, T beta, CT* C,
+                                                   int64_t ldc, int upper) {
   const int64_t m0 = static_cast<int64_t>(blockIdx.y) * TM;
   const int64_t n0 = static_cast<int64_t>(blockIdx.x) * TN;
   if (upper && n0 + TN - 1 < m0) return;
 
-  __shared__ __align__(16) float As[2][TK][TM + PAD];
-  __shared__ __align__(16) float Bs[2][TK][TN + PAD];
+  __shared__ __align__(16) T As[2][TK][TM + PAD];
+  __shared__ __align__(16) T Bs[2][TK][TN + PAD];
   const int tid = threadIdx.x;
   const int tx = tid & 15, ty = tid >> 4;
 
-  float ra[4], rb[4];
+  T ra[4], rb[4];
   auto load_regs = [&](int64_t k0) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int e = tid + 256 * i;
       const int am = e >> 3, ak = e & 7;
       const int64_t gm = m0 + am, gk = k0 + ak;
-      ra[i] = (gm < M && gk < K) ? A[gm * lda + gk] : 0.f;
+      ra[i] = (gm < M && gk < K) ? A[gm * lda + gk] : T(0);
       if (TRANSB) {
         const int bn = e >> 3, bk = e & 7;
         const int64_t gn = n0 + bn, gk2 = k0 + bk;
-        rb[i] = (gn < N && gk2 < K) ? B[gn * ldb + gk2] : 0.f;
+        rb[i] = (gn < N && gk2 < K) ? B[gn * ldb + gk2] : T(0);
       } else {
         const int bk = e >> 7, bn = e & 127;
         const int64_t gn = n0 + bn, gk2 = k0 + bk;
-        rb[i] = (gn < N && gk2 < K) ? B[gk2 * ldb + gn] : 0.f;
+        rb[i] = (gn < N && gk2 < K) ? B[gk2 * ldb + gn] : T(0);
       }
     }
   };
@@ -60,11 +59,11 @@ __global__ void __launch_bounds__(256) sgemm_kernel(int64_t M, int64_t N, int64_
     }
   };
 
-  float acc[8][8];
+  T acc[8][8];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    for (int j = 0; j < 8; ++j) acc[i][j] = T(0);
 
   const int64_t nkt = (K + TK - 1) / TK;
   int buf = 0;
@@ -77,16 +76,18 @@ __global__ void __launch_bounds__(256) sgemm_kernel(int64_t M, int64_t N, int64_
     if (kt + 1 < nkt) load_regs((kt + 1) * TK);
 #pragma unroll
     for (int k = 0; k < TK; ++k) {
-      const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][k][ty * 4]);
-      const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][k][64 + ty * 4]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][k][tx * 4]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][k][64 + tx * 4]);
-      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+      T a[8], b[8];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        a[q] = As[buf][k][ty * 4 + q];
+        a[4 + q] = As[buf][k][64 + ty * 4 + q];
+        b[q] = Bs[buf][k][tx * 4 + q];
+        b[4 + q] = Bs[buf][k][64 + tx * 4 + q];
+      }
 #pragma unroll
       for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        for (int j = 0; j < 8; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
     }
     if (kt + 1 < nkt) store_smem(buf ^ 1);
     __syncthreads();
@@ -101,9 +102,12 @@ __global__ void __launch_bounds__(256) sgemm_kernel(int64_t M, int64_t N, int64_
     for (int j = 0; j < 8; ++j) {
       const int64_t gn = n0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + (j - 4));
       if (gn >= N) continue;
-      float* cp = C + gm * ldc + gn;
-      const float v = alpha * acc[i][j];
-      *cp = (beta == 0.f) ? v : fmaf(beta, *cp, v);
+      CT* cp = C + gm * ldc + gn;
+      const T v = alpha * acc[i][j];
+      if constexpr (sizeof(CT) > sizeof(T))
+        *cp = *cp + static_cast<CT>(v);  // fp32 product, fp64 running value
+      else
+        *cp = (beta == T(0)) ? v : fma(beta, *cp, v);
     }
   }
 }
@@ -116,9 +120,30 @@ int sgemm(cudaStream_t s, int64_t M, int64_t N, int64_t K, float alpha, const fl
   dim3 grid(static_cast<unsigned>((N + TN - 1) / TN), static_cast<unsigned>((M + TM - 1) / TM));
   if (grid.y > 65535u) return GPTQ_ERR_UNSUPPORTED;
   if (transB)
-    sgemm_kernel<true><<<grid, 256, 0, s>>>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc, upper ? 1 : 0);
+    gemm_kernel<float, true, float><<<grid, 256, 0, s>>>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc, upper ? 1 : 0);
   else
-    sgemm_kernel<false><<<grid, 256, 0, s>>>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc, upper ? 1 : 0);
+    gemm_kernel<float, false, float><<<grid, 256, 0, s>>>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc, upper ? 1 : 0);
+  return after_launch();
+}
+
+int dgemm(cudaStream_t s, int64_t M, int64_t N, int64_t K, double alpha, const double* A, int64_t lda,
+          const double* B, int64_t ldb, bool transB, double beta, double* C, int64_t ldc, bool upper) {
+  if (M <= 0 || N <= 0) return GPTQ_OK;
+  dim3 grid(static_cast<unsigned>((N + TN - 1) / TN), static_cast<unsigned>((M + TM - 1) / TM));
+  if (grid.y > 65535u) return GPTQ_ERR_UNSUPPORTED;
+  if (transB)
+    gemm_kernel<double, true, double><<<grid, 256, 0, s>>>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc, upper ? 1 : 0);
+  else
+    gemm_kernel<double, false, double><<<grid, 256, 0, s>>>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc, upper ? 1 : 0);
+  return after_launch();
+}
+
+int sgemm_acc64(cudaStream_t s, int64_t M, int64_t N, int64_t K, float alpha, const float* A, int64_t lda,
+                const float* B, int64_t ldb, double* C, int64_t ldc) {
+  if (M <= 0 || N <= 0) return GPTQ_OK;
+  dim3 grid(static_cast<unsigned>((N + TN - 1) / TN), static_cast<unsigned>((M + TM - 1) / TM));
+  if (grid.y > 65535u) return GPTQ_ERR_UNSUPPORTED;
+  gemm_kernel<float, false, double><<<grid, 256, 0, s>>>(M, N, K, alpha, A, lda, B, ldb, 1.f, C, ldc, 0);
   return after_launch();
 }
 

@@ -13,12 +13,17 @@
 //   quantized its slot holds err_j, so the lazy updates read the errors in place.
 // * codesT [n_in, n_out] uint8 holds the codes in sweep order (column-major w.r.t. W),
 //   so both the sweep's writes and the packer's reads are coalesced across rows.
-// * Panels of P <= 128 columns: one kernel per panel, rows in parallel (8 threads per
-//   row, 16 columns per thread in registers, the panel's block of U in shared memory,
+// * Panels of P <= 64 columns: one kernel per panel, rows in parallel (16 threads per
+//   row, 4 columns per thread in registers, the panel's block of U in shared memory,
 //   group min/max and the error broadcast via warp shuffles).
+// * Precision: the running weights, the errors, U and the lazy-update products are all
+//   fp64; only the code decision (w / s, rounding) is taken in fp32.  GPTQ's sweep is a
+//   long chain of rounding decisions, each depending on every earlier error of its row,
+//   so fp32-level perturbations of the running weights grow into different codes over
+//   thousands of columns.
 // * Two-level lazy updates: after each panel its errors update the rest of the current
-//   outer block (<= 1024 columns, L2-resident); after each outer block its errors update
-//   every later column in one GEMM with K = outer block width.
+//   outer block (<= 1024 columns); after each outer block its errors update every later
+//   column in one GEMM with K = outer block width.
 #include <algorithm>
 
 #include "common.cuh"
@@ -26,11 +31,13 @@
 namespace gptq {
 namespace {
 
-constexpr int PW = 128;                // max panel width
-constexpr int TPR = 8;                 // threads per row
+constexpr int PW = 64;                 // max panel width
+constexpr int TPR = 16;                // threads per row
 constexpr int NCOL = PW / TPR;         // columns per thread
 constexpr int ROWS = 256 / TPR;        // rows per CTA
-constexpr int PANEL_SMEM = PW * PW * 4 + PW * ROWS;
+// U block (fp64) + per-column reciprocal pivots (fp64) + per-column group parameters of
+// every row (scale fp32, zero int32) + codes.
+constexpr int PANEL_SMEM = PW * PW * 8 + PW * 8 + PW * ROWS * 8 + PW * ROWS;
 
 // ---------------------------------------------------------------- quantizer (float32 decisions)
 __device__ __forceinline__ void params_sym(float amax, int bits, float& s, int& z) {
@@ -72,12 +79,12 @@ __device__ __forceinline__ int64_t clamp_idx(int32_t v, int64_t n) {
 // ---------------------------------------------------------------- staging kernels
 template <typename T>
 __global__ void stage_weights_kernel(const T* __restrict__ W, int64_t n_out, int64_t n_in,
-                                     const int32_t* __restrict__ perm, float* __restrict__ Wk) {
+                                     const int32_t* __restrict__ perm, double* __restrict__ Wk) {
   const int64_t o = blockIdx.y;
   for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < n_in;
        j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t c = perm ? clamp_idx(perm[j], n_in) : j;
-    Wk[o * n_in + j] = to_f32(W[o * n_in + c]);
+    Wk[o * n_in + j] = static_cast<double>(to_f32(W[o * n_in + c]));
   }
 }
 
@@ -113,7 +120,7 @@ __global__ void fixed_params_kernel(const T* __restrict__ W, int64_t n_out, int6
 
 // Non-static groups wider than a panel: parameters from the current (error-updated)
 // weights of sweep columns [j0, j0 + gsz) when the sweep reaches j0.  One warp per row.
-__global__ void current_params_kernel(const float* __restrict__ Wk, int64_t n_out, int64_t n_in, int64_t j0,
+__global__ void current_params_kernel(const double* __restrict__ Wk, int64_t n_out, int64_t n_in, int64_t j0,
                                       int gsz, int bits, int sym, float* __restrict__ scales,
                                       int32_t* __restrict__ zeros) {
   const int64_t o = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -121,7 +128,7 @@ __global__ void current_params_kernel(const float* __restrict__ Wk, int64_t n_ou
   if (o >= n_out) return;
   float mn = INFINITY, mx = -INFINITY;
   for (int64_t c = j0 + lane; c < j0 + gsz; c += 32) {
-    const float v = Wk[o * n_in + c];
+    const float v = static_cast<float>(Wk[o * n_in + c]);
     mn = fminf(mn, v);
     mx = fmaxf(mx, v);
   }
@@ -140,9 +147,10 @@ __global__ void current_params_kernel(const float* __restrict__ Wk, int64_t n_ou
 
 // ---------------------------------------------------------------- panel kernel
 struct PanelArgs {
-  float* Wk;
+  double* Wk;
+  double* Err;
   int64_t n_out, n_in;
-  const float* U;
+  const double* U;
   int64_t j0;
   int pw;
   int bits, gsz;
@@ -158,8 +166,11 @@ struct PanelArgs {
 
 __global__ void __launch_bounds__(256) sweep_panel_kernel(PanelArgs a) {
   extern __shared__ __align__(16) unsigned char psm[];
-  float* Us = reinterpret_cast<float*>(psm);               // [PW][PW], U[j0 + r][j0 + c]
-  uint8_t* cs = reinterpret_cast<uint8_t*>(Us + PW * PW);  // [PW][ROWS] codes of this CTA
+  double* Us = reinterpret_cast<double*>(psm);               // [PW][PW], U[j0 + r][j0 + c]
+  double* rdiag = reinterpret_cast<double*>(Us + PW * PW);   // [PW], 1 / U[j][j]
+  float* ps = reinterpret_cast<float*>(rdiag + PW);          // [PW][ROWS] scale per column and row
+  int* pz = reinterpret_cast<int*>(ps + PW * ROWS);          // [PW][ROWS] zero point
+  uint8_t* cs = reinterpret_cast<uint8_t*>(pz + PW * ROWS);  // [PW][ROWS] codes of this CTA
   const int tid = threadIdx.x, lane = tid & 31;
   const int tsub = tid % TPR;
   const int rloc = tid / TPR;
@@ -174,19 +185,35 @@ __global__ void __launch_bounds__(256) sweep_panel_kernel(PanelArgs a) {
 
   for (int e = tid; e < PW * PW; e += 256) {
     const int r = e / PW, c = e % PW;
-    Us[e] = (r < pw && c < pw && c >= r) ? a.U[(j0 + r) * n_in + j0 + c] : 0.f;
+    Us[e] = (r < pw && c < pw && c >= r) ? a.U[(j0 + r) * n_in + j0 + c] : 0.0;
   }
-  float v[NCOL];
+  // Parameters fixed before this panel (static groups, group_size -1, or groups wider
+  // than the panel): stage them per column so the serial chain below never waits on
+  // global memory.
+  if (!a.in_panel_params) {
+    for (int c = tsub; c < pw; c += TPR) {
+      const int64_t j = j0 + c;
+      int64_t g = 0;
+      if (a.gsz > 0) g = (a.static_groups && a.perm) ? clamp_idx(a.perm[j], n_in) / a.gsz : j / a.gsz;
+      ps[c * ROWS + rloc] = active ? a.scales[g * n_out + row] : 1.f;
+      pz[c * ROWS + rloc] = active ? a.zeros[g * n_out + row] : 0;
+    }
+  }
+  // The panel's running weights live in registers in fp64: each column of the panel
+  // receives up to PW-1 compensation updates here, and rounding the running value to
+  // fp32 after each of them would push near-tie codes across a rounding boundary.
+  double v[NCOL];
 #pragma unroll
   for (int m = 0; m < NCOL; ++m) {
     const int col = tsub + TPR * m;
-    v[m] = (active && col < pw) ? a.Wk[row * n_in + j0 + col] : 0.f;
+    v[m] = (active && col < pw) ? a.Wk[row * n_in + j0 + col] : 0.0;
   }
+  __syncthreads();
+  if (tid < pw) rdiag[tid] = 1.0 / Us[tid * PW + tid];
   __syncthreads();
 
   float s = 1.f;
   int z = 0;
-  int64_t cur_g = -1;
   double lsum = 0.0;
 
 #pragma unroll
@@ -200,8 +227,9 @@ __global__ void __launch_bounds__(256) sweep_panel_kernel(PanelArgs a) {
           for (int m = c / TPR; m < NCOL; ++m) {
             const int col = tsub + TPR * m;
             if (col >= c && col < c + a.gsz) {
-              mn = fminf(mn, v[m]);
-              mx = fmaxf(mx, v[m]);
+              const float x = static_cast<float>(v[m]);
+              mn = fminf(mn, x);
+              mx = fmaxf(mx, x);
             }
           }
 #pragma unroll
@@ -215,44 +243,38 @@ __global__ void __launch_bounds__(256) sweep_panel_kernel(PanelArgs a) {
             a.zeros[(j / a.gsz) * n_out + row] = z;
           }
         }
-      } else {
-        int64_t g = 0;
-        if (a.gsz > 0) g = (a.static_groups && a.perm) ? clamp_idx(a.perm[j], n_in) / a.gsz : j / a.gsz;
-        if (g != cur_g) {
-          cur_g = g;
-          if (active) {
-            s = a.scales[g * n_out + row];
-            z = a.zeros[g * n_out + row];
-          }
-        }
       }
-      float err = 0.f;
+      double err = 0.0;
       if (tsub == (c % TPR)) {
-        const float w = v[c / TPR];
-        const int q = quant_code(w, s, z, maxq);
-        const float what = __fmul_rn(s, static_cast<float>(q - z));
-        err = __fdiv_rn(__fsub_rn(w, what), Us[c * PW + c]);
+        if (!a.in_panel_params) {
+          s = ps[c * ROWS + rloc];
+          z = pz[c * ROWS + rloc];
+        }
+        const double w = v[c / TPR];
+        const int q = quant_code(static_cast<float>(w), s, z, maxq);
+        const double what = static_cast<double>(s) * static_cast<double>(q - z);
+        err = (w - what) * rdiag[c];
         v[c / TPR] = err;
         cs[c * ROWS + rloc] = static_cast<uint8_t>(q);
-        lsum += static_cast<double>(err) * err;
+        lsum += err * err;
       }
       err = __shfl_sync(FULL, err, base_lane + (c % TPR));
 #pragma unroll
       for (int m = c / TPR; m < NCOL; ++m) {
         const int col = tsub + TPR * m;
-        if (col > c) v[m] = fmaf(-err, Us[c * PW + col], v[m]);
+        if (col > c) v[m] = fma(-err, Us[c * PW + col], v[m]);
       }
     }
   }
 
-  // errors back into the working copy (they feed the lazy updates)
+  // errors feed the lazy updates of the later columns
 #pragma unroll
   for (int m = 0; m < NCOL; ++m) {
     const int col = tsub + TPR * m;
-    if (active && col < pw) a.Wk[row * n_in + j0 + col] = v[m];
+    if (active && col < pw) a.Err[row * n_in + j0 + col] = v[m];
   }
   __syncthreads();
-  // codes: one 32-byte row segment per column
+  // codes: one ROWS-byte row segment per column
   for (int e = tid; e < pw * ROWS; e += 256) {
     const int c = e / ROWS, r = e % ROWS;
     if (row0 + r < n_out) a.codesT[(j0 + c) * n_out + row0 + r] = cs[c * ROWS + r];
@@ -385,6 +407,7 @@ int run_sweep(SweepArgs& a, cudaStream_t s, int* panel_width, int* outer_width) 
 
   PanelArgs pa;
   pa.Wk = a.Wk;
+  pa.Err = a.Err;
   pa.n_out = n_out;
   pa.n_in = n_in;
   pa.U = a.U;
@@ -414,11 +437,11 @@ int run_sweep(SweepArgs& a, cudaStream_t s, int* panel_width, int* outer_width) 
       sweep_panel_kernel<<<panel_grid, 256, PANEL_SMEM, s>>>(pa);
       GPTQ_TRY(after_launch());
       if (p1 < O1)  // rest of the outer block: W[:, p1:O1] -= Err[:, p0:p1] U[p0:p1, p1:O1]
-        GPTQ_TRY(sgemm(s, n_out, O1 - p1, p1 - p0, -1.f, a.Wk + p0, n_in, a.U + p0 * n_in + p1, n_in, false, 1.f,
+        GPTQ_TRY(dgemm(s, n_out, O1 - p1, p1 - p0, -1.0, a.Err + p0, n_in, a.U + p0 * n_in + p1, n_in, false, 1.0,
                        a.Wk + p1, n_in, false));
     }
     if (O1 < n_in)  // every later column: W[:, O1:] -= Err[:, O0:O1] U[O0:O1, O1:]
-      GPTQ_TRY(sgemm(s, n_out, n_in - O1, O1 - O0, -1.f, a.Wk + O0, n_in, a.U + O0 * n_in + O1, n_in, false, 1.f,
+      GPTQ_TRY(dgemm(s, n_out, n_in - O1, O1 - O0, -1.0, a.Err + O0, n_in, a.U + O0 * n_in + O1, n_in, false, 1.0,
                      a.Wk + O1, n_in, false));
   }
   if (a.stats) GPTQ_CUDA(cudaEventRecord(a.ev[2], s));

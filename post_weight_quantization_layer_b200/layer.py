@@ -1,0 +1,87 @@
+"""Decoder-layer driver: quantize every linear of one transformer block.
+
+The modules that read the same input share one calibration Hessian (q/k/v the
+attention input, gate/up the MLP input; the OLMo quick-start's fused att_proj,
+§六 6.1).  Each distinct Hessian is accumulated once, factored once
+(gptq_factor_hessian), and every module that reads it is swept against that
+factor (gptq_quantize_layer_factored).  All arithmetic runs in the native
+library; this module only sequences the calls and records per-phase CUDA-event
+times on the stream.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import torch
+
+from . import api
+
+
+@dataclass
+class LayerTimes:
+    hessian_ms: float = 0.0
+    factor_ms: float = 0.0
+    sweep_ms: float = 0.0
+    hessian_launch_ms: list = field(default_factory=list)
+
+    @property
+    def total_ms(self):
+        return self.hessian_ms + self.factor_ms + self.sweep_ms
+
+
+def quantize_decoder_layer(acts, weights, modules, qcfg, hessians=None, timing=False, stream=None):
+    """Quantize the linears of one decoder layer.
+
+    acts:     {h_index: X [tokens, n] fp16/bf16 CUDA tensor, or a list of token chunks}
+    weights:  {module name: W [n_out, n_in] CUDA tensor}
+    modules:  iterable of objects with .name and .h_index
+    qcfg:     object with bits, group_size, damp_percent, sym, desc_act, static_groups, blocksize
+    hessians: optional {h_index: preallocated [n, n] fp32 CUDA tensor} (zeroed here)
+    Returns ({module name: QuantResult}, LayerTimes or None).
+    """
+    stream = stream or torch.cuda.current_stream()
+    ev = (lambda: torch.cuda.Event(enable_timing=True)) if timing else None
+    times = LayerTimes() if timing else None
+    marks = []
+
+    def mark():
+        if timing:
+            e = ev()
+            e.record(stream)
+            marks.append(e)
+            return e
+        return None
+
+    with torch.cuda.stream(stream):
+        mark()
+        Hs = {}
+        launch_marks = []
+        for h, X in acts.items():
+            chunks = X if isinstance(X, (list, tuple)) else [X]
+            n = chunks[0].shape[1]
+            H = hessians[h] if hessians is not None else torch.empty(n, n, dtype=torch.float32, device=chunks[0].device)
+            H.zero_()
+            a = mark()
+            for c in chunks:
+                api.accumulate_hessian(c, H, stream=stream)
+            b = mark()
+            launch_marks.append((a, b))
+            Hs[h] = H
+        m_h = mark()
+        factors = {h: api.factor_hessian(H, qcfg.damp_percent, qcfg.desc_act, stream=stream) for h, H in Hs.items()}
+        m_f = mark()
+        results = {}
+        for mod in modules:
+            U, perm = factors[mod.h_index]
+            results[mod.name] = api.quantize_layer_factored(
+                weights[mod.name], U, perm, qcfg.bits, qcfg.group_size, qcfg.sym, qcfg.static_groups,
+                qcfg.blocksize, stream=stream)
+        m_s = mark()
+    if timing:
+        m_s.synchronize()
+        times.hessian_ms = marks[0].elapsed_time(m_h)
+        times.factor_ms = m_h.elapsed_time(m_f)
+        times.sweep_ms = m_f.elapsed_time(m_s)
+        times.hessian_launch_ms = [a.elapsed_time(b) for a, b in launch_marks]
+    return results, times

@@ -32,12 +32,12 @@ def test_factor_matches_oracle(n, T, desc_act):
     Ug = U.cpu().double().numpy()
     assert np.all(np.tril(Ug, -1) == 0)
     assert np.all(np.diag(Ug) > 0)
-    # row-relative error of the compensation coefficients
+    # row-relative error of the compensation coefficients: the GPU factor works in fp64
+    # from the same fp32 Hessian, so only fp64 rounding (times the condition number) remains
     err = np.abs(Ug - U_ref).max(axis=1) / np.abs(U_ref).max(axis=1)
-    assert err.max() < 2e-3, err.max()
-    # U^T U H_d = I up to fp32 factorisation error
+    assert err.max() < 1e-7, err.max()
     R = Ug.T @ Ug @ Hd - np.eye(n)
-    assert np.abs(R).max() < 5e-3
+    assert np.abs(R).max() < 1e-7
 
 
 def test_not_positive_definite_is_reported():
@@ -52,7 +52,8 @@ def test_not_positive_definite_is_reported():
     # the context stays usable after the error
     U, _ = gq.factor_hessian(torch.eye(64, device=dev) * 2, 0.01)
     torch.cuda.synchronize()
-    assert torch.allclose(torch.diag(U).cpu(), torch.full((64,), (1 / 2.02) ** 0.5), rtol=1e-6)
+    assert torch.allclose(torch.diag(U).cpu(), torch.full((64,), (1 / 2.02) ** 0.5, dtype=torch.float64),
+                          rtol=1e-12)
 
 
 def test_act_order_ties_are_stable():

@@ -89,7 +89,7 @@ def test_factored_sweep_with_oracle_factor():
     perm = O.act_order_perm(Hn)
     U = O.inverse_cholesky_upper(O.dampen(Hn[np.ix_(perm, perm)], 0.01))
     dev = device()
-    res = gq.quantize_layer_factored(W.to(dev), torch.from_numpy(U).float().to(dev),
+    res = gq.quantize_layer_factored(W.to(dev), torch.from_numpy(U).to(dev),
                                      torch.from_numpy(perm.astype(np.int32)).to(dev), 4, 64, True, False, 128)
     torch.cuda.synchronize()
     ref = O.gptq_quantize(W.double().numpy(), Hn, 4, 64, 0.01, True, True, False)
@@ -125,3 +125,13 @@ def test_not_pd_through_quantize_layer():
     with pytest.raises(gq.GPTQError) as e:
         gq.quantize_layer(W, torch.zeros(64, 64, device=dev), 4, 32)
     assert e.value.status == 3
+
+
+def test_trim_workspace_keeps_library_usable():
+    from post_weight_quantization_layer_b200 import _native
+    dev = device()
+    W, H = _problem(32, 128, 512, 8)
+    a = gq.quantize_layer(W.to(dev), H.to(dev), 4, 32)
+    assert _native.lib().gptq_trim_workspace() == 0
+    b = gq.quantize_layer(W.to(dev), H.to(dev), 4, 32)
+    assert torch.equal(a.qweight, b.qweight)
