@@ -153,6 +153,31 @@ int gptq_quantize_layer_factored(const void* W, int w_dtype, int64_t n_out, int6
                                  int32_t* g_idx, void* stream, gptq_stats* stats);
 
 /*
+ * gptq_factor_hessian for callers that cannot allocate device memory.
+ * The paper has no counterpart: this is a deployment variant of the factor call.
+ *
+ * Who needs it: code that runs where every device allocation is forbidden or owned by
+ * someone else - an inference or serving runtime that reserves a fixed arena at
+ * start-up, a real-time loop that must not call an allocator, a plugin whose host caps
+ * the allocator.  gptq_factor_hessian takes its workspace from a memory pool; this
+ * variant runs the same kernels with the same arguments, outputs and results, but its
+ * scratch is one fixed array of device memory built into the library (about 8.9 MB,
+ * held on every GPU that loads the library until the process exits).  It calls no
+ * cudaMalloc, cudaFree or other allocating routine.
+ *
+ * Limits and rules:
+ * - n_in <= 1024 (and a multiple of 8); larger sizes return GPTQ_ERR_UNSUPPORTED.
+ * - The first call on a device looks up the array's device address on that device
+ *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ * - All calls share the one array and it keeps the last call's contents; calls that
+ *   may overlap on the GPU (different streams, different host threads) race and must be
+ *   serialised by the caller.
+ * Blocking, like gptq_factor_hessian.
+ */
+int gptq_factor_hessian_noalloc(const float* H, int64_t n_in, float damp_percent, int desc_act,
+                                double* U, int32_t* perm, void* stream);
+
+/*
  * Release the device memory that the library's workspace pool keeps cached between
  * calls on the current device (workspace is allocated stream-ordered from a pool owned
  * by the library and reused across calls).  Synchronises the device first.
