@@ -161,7 +161,7 @@ int gptq_quantize_layer_factored(const void* W, int w_dtype, int64_t n_out, int6
  * start-up, a real-time loop that must not call an allocator, a plugin whose host caps
  * the allocator.  gptq_factor_hessian takes its workspace from a memory pool; this
  * variant runs the same kernels with the same arguments, outputs and results, but its
- * scratch is one fixed array of device memory built into the library (about 8.9 MB,
+ * scratch is one fixed array of device memory built into the library (about 13.3 MB,
  * held on every GPU that loads the library until the process exits).  It calls no
  * cudaMalloc, cudaFree or other allocating routine.
  *

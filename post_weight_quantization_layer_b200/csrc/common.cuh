@@ -71,9 +71,14 @@ int sgemm(cudaStream_t s, int64_t M, int64_t N, int64_t K, float alpha, const fl
 // C[m,n] = C[m,n] + (double)(alpha * sum_k A[m,k] B(k,n)).
 int sgemm_acc64(cudaStream_t s, int64_t M, int64_t N, int64_t K, float alpha, const float* A, int64_t lda,
                 const float* B, int64_t ldb, double* C, int64_t ldc);
-// fp64 operands, fp64 accumulation (same conventions as sgemm).
+// fp64 operands, fp64 accumulation (same conventions as sgemm).  `tri` declares operands
+// that are triangular with exact zeros elsewhere, so that those K ranges are skipped:
+constexpr int kTriAUpper = 1;   // A(m,k) == 0 for k < m
+constexpr int kTriBUpper = 2;   // B(k,n) == 0 for k > n   (op(B) upper triangular)
+constexpr int kTriBTUpper = 4;  // B(k,n) == 0 for k < n   (op(B) = U^T with U upper)
 int dgemm(cudaStream_t s, int64_t M, int64_t N, int64_t K, double alpha, const double* A, int64_t lda,
-          const double* B, int64_t ldb, bool transB, double beta, double* C, int64_t ldc, bool upper);
+          const double* B, int64_t ldb, bool transB, double beta, double* C, int64_t ldc, bool upper,
+          int tri = 0);
 
 // factor.cu: U (sweep order, fp64) and perm from H.  `work` holds factor_work_bytes(n),
 // `small` factor_small_bytes(n); `status` is a device int.

@@ -10,10 +10,17 @@
 // Route: instead of inverting and then factoring (about 5n^3/3 flops), factor the
 // damped Hessian from the bottom-right corner, H_d = V V^T with V upper triangular,
 // and invert V: inverse(H_d) = V^-T V^-1, so U = V^-1 is exactly the upper factor
-// with inverse(H_d) = U^T U and a positive diagonal (2n^3/3 flops).  Both steps are
-// blocked with 64-wide blocks: a single-CTA kernel factors and inverts each diagonal
-// block in shared memory (and checks every pivot), and the off-diagonal work runs as
-// GEMMs.
+// with inverse(H_d) = U^T U and a positive diagonal (2n^3/3 flops).
+//
+// Both are done together, recursively.  Split H_d = [[A, B], [B^T, C]] with the larger,
+// NB-aligned part C at the bottom right.  Then, with C = V22 V22^T and U22 = V22^-1:
+//   P   = B U22^T              (the off-diagonal block V12 of V)
+//   A' := A - P P^T            (Schur complement; upper triangle only)
+//   T   = P U22
+//   U11 = factor-and-invert(A'),  U12 = -U11 T,
+// since V^-1 = [[V11^-1, -V11^-1 V12 V22^-1], [0, V22^-1]].  Blocks of at most NB = 128 are
+// factored and inverted by one CTA in shared memory (which also checks every pivot);
+// everything else is four large GEMMs per level.  V itself is never stored.
 //
 // Precision: the factorisation runs in fp64 and U stays fp64.  The forward error of a
 // Cholesky factor grows like cond(H_d) times the working precision; with cond(H_d) ~ 1e4
@@ -21,15 +28,17 @@
 // in U, and a sweep over thousands of columns amplifies even fp32 rounding of U into
 // different codes.
 #include <algorithm>
+#include <vector>
 
 #include "common.cuh"
 
 namespace gptq {
 namespace {
 
-constexpr int NB = 64;  // block width of the factorisation
+constexpr int NB = 128;  // leaf block width of the factorisation
 constexpr int DIAG_THREADS = 512;
 constexpr int SP = NB + 1;  // padded pitch of the diagonal block in shared memory
+constexpr int TP = NB / 2 + 1;
 using real = double;     // working precision of the factorisation
 
 // Sum of diag(H) in double.
@@ -86,132 +95,251 @@ __global__ void permute_damp_kernel(const float* __restrict__ H, int64_t n, cons
   A[i * n + j] = v;
 }
 
-// Factor the diagonal block A[k0:k0+nb, k0:k0+nb] (upper part valid) as V V^T with V upper,
-// write V back into A, and its inverse into Winv[k0:k0+nb, 0:nb] (ld NB).  A pivot that is
-// not positive and finite sets *status = NOT_PD; the factorisation continues with a unit
-// pivot so that every later kernel still sees finite numbers.
+// Factor the diagonal block A[k0:k0+nb, k0:k0+nb] (upper part valid) as V V^T with V upper
+// and write its inverse into R[k0:k0+nb, k0:k0+nb] (same leading dimension, zeros below the
+// diagonal).  A pivot that is not positive and finite sets *status = NOT_PD; the
+// factorisation continues with a unit pivot so that every later kernel still sees finite
+// numbers.
 //
 // The block is padded to NB x NB with an identity in its bottom-right corner (no coupling),
 // which leaves the real part of V and V^-1 unchanged and lets every size use the same
-// power-of-two inverse below.
-__global__ void __launch_bounds__(DIAG_THREADS) chol_diag_kernel(real* A, int64_t lda, int64_t k0, int nb,
-                                                                 real* Winv, int* status) {
+// power-of-two inverse below.  Everything happens in place in shared memory: S holds the
+// block, then V, then V^-1.
+__global__ void __launch_bounds__(DIAG_THREADS) chol_diag_kernel(const real* A, int64_t lda, int64_t k0, int nb,
+                                                                 real* R, int* status) {
   extern __shared__ real sm[];
-  real* S = sm;              // V, [NB][SP]
-  real* X = sm + NB * SP;    // V^-1, [NB][SP]
-  real* T = X + NB * SP;     // product scratch, [NB/2][SP]
-  real* col = T + (NB / 2) * SP;  // scaled column, [NB]
+  real* S = sm;                         // [NB][SP]
+  real* T = S + NB * SP;                // [NB/2][TP] product scratch
+  real* col = T + (NB / 2) * TP;        // [NB] scaled column
+  real* rdiag = col + NB;               // [NB] 1 / V[j][j]
+  real* blk = rdiag + NB;               // [NB/16][16][17] copies of the 16x16 diagonal blocks
   __shared__ int bad;
+  __shared__ real colbuf[2][NB];        // column c of the running matrix, double-buffered
   const int tid = threadIdx.x;
   if (tid == 0) bad = 0;
-  for (int e = tid; e < NB * NB; e += DIAG_THREADS) {
-    const int i = e / NB, j = e % NB;
-    real v = 0;
-    if (i < nb && j < nb) {
-      if (i <= j) v = A[(k0 + i) * lda + k0 + j];
-    } else if (i == j) {
-      v = 1;
-    }
-    S[i * SP + j] = v;
-    X[i * SP + j] = 0;
-  }
-  // Each thread owns fixed elements (i <= j) of the upper triangle for the rank-1 updates.
-  constexpr int NUP = NB * (NB + 1) / 2;
-  constexpr int SLOTS = (NUP + DIAG_THREADS - 1) / DIAG_THREADS;
-  int own[SLOTS];
+  // Register blocking: thread (rb, cb) holds rows 4rb..4rb+3 x cols 8cb..8cb+7 of the block
+  // (upper triangle; the identity pads it to NB x NB).
+  const int rb = tid >> 4, cb = tid & 15;
+  const int i0 = rb * 4, j0 = cb * 8;
+  real r[4][8];
 #pragma unroll
-  for (int r = 0; r < SLOTS; ++r) {
-    int e = tid + r * DIAG_THREADS, i = 0;
-    if (e < NUP) {
-      while (e >= NB - i) {
-        e -= NB - i;
-        ++i;
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+      const int i = i0 + a, j = j0 + b;
+      real v = 0;
+      if (i <= j) {
+        if (j < nb)
+          v = A[(k0 + i) * lda + k0 + j];
+        else if (i == j)
+          v = 1;
       }
-      own[r] = (i << 8) | (i + e);
-    } else {
-      own[r] = -1;
+      r[a][b] = v;
     }
-  }
-  __syncthreads();
+  // Reverse Cholesky: for c = NB-1 .. 0, V[c][c] = sqrt(S[c][c]), V[i][c] = S[i][c] / V[c][c]
+  // for i < c, then S[i][j] -= V[i][c] V[j][c] for i <= j < c.
   for (int c = NB - 1; c >= 0; --c) {
-    real d = S[c * SP + c];
+    real* cb_buf = colbuf[c & 1];
+    if (cb == (c >> 3)) {
+#pragma unroll
+      for (int b = 0; b < 8; ++b)
+        if (j0 + b == c) {
+#pragma unroll
+          for (int a = 0; a < 4; ++a)
+            if (i0 + a <= c) cb_buf[i0 + a] = r[a][b];
+        }
+    }
+    __syncthreads();
+    real d = cb_buf[c];
     if (!(d > 0) || !isfinite(d)) {
       if (tid == 0) bad = 1;
       d = 1;
     }
     const real v = sqrt(d);
-    if (tid < c) col[tid] = S[tid * SP + c] / v;
-    __syncthreads();
-    if (tid == 0) S[c * SP + c] = v;
-    if (tid < c) S[tid * SP + c] = col[tid];
+    const real rv = 1 / v;
+    if (j0 < c && i0 < c) {
+      real ci[4], cj[8];
 #pragma unroll
-    for (int r = 0; r < SLOTS; ++r) {
-      const int o = own[r];
-      const int i = o >> 8, j = o & 255;
-      if (o >= 0 && j < c) S[i * SP + j] = fma(-col[i], col[j], S[i * SP + j]);
+      for (int a = 0; a < 4; ++a) ci[a] = cb_buf[min(i0 + a, c)] * rv;
+#pragma unroll
+      for (int b = 0; b < 8; ++b) cj[b] = cb_buf[min(j0 + b, c)] * rv;
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b)
+          if (i0 + a <= j0 + b && j0 + b < c) r[a][b] = fma(-ci[a], cj[b], r[a][b]);
     }
-    __syncthreads();
+    if (cb == (c >> 3)) {  // finish column c of V in registers
+#pragma unroll
+      for (int b = 0; b < 8; ++b)
+        if (j0 + b == c) {
+#pragma unroll
+          for (int a = 0; a < 4; ++a) {
+            if (i0 + a < c) r[a][b] *= rv;
+            if (i0 + a == c) r[a][b] = v;
+          }
+        }
+    }
+    if (tid == 0) rdiag[c] = rv;
   }
+  // V to shared memory for the inverse
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 8; ++b) S[(i0 + a) * SP + j0 + b] = r[a][b];
+  __syncthreads();
 
-  // X = V^-1 by doubling: invert 16x16 diagonal blocks, then join neighbours with
+  // V^-1 in place by doubling: invert the 16x16 diagonal blocks, then join neighbours with
   // [[A, B], [0, C]]^-1 = [[A^-1, -A^-1 B C^-1], [0, C^-1]].
   {
     const int warp = tid >> 5, lane = tid & 31;
-    if (warp < NB / 16 && lane < 16) {
-      const int p = warp * 16, j = p + lane;
-      X[j * SP + j] = 1 / S[j * SP + j];
-      for (int i = j - 1; i >= p; --i) {
-        real acc = 0;
-        for (int l = i + 1; l <= j; ++l) acc = fma(S[i * SP + l], X[l * SP + j], acc);
-        X[i * SP + j] = -acc / S[i * SP + i];
+    if (warp < NB / 16) {
+      const int p = warp * 16;
+      real* b = blk + warp * 16 * 17;
+      for (int e = lane; e < 256; e += 32) b[(e >> 4) * 17 + (e & 15)] = S[(p + (e >> 4)) * SP + p + (e & 15)];
+      __syncwarp();
+      if (lane < 16) {
+        const int j = lane;
+        real x[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) x[i] = (i == j) ? rdiag[p + i] : real(0);
+#pragma unroll
+        for (int i = 15; i >= 0; --i) {
+          if (i < j) {
+            real acc = 0;
+#pragma unroll
+            for (int l = i + 1; l < 16; ++l)
+              if (l <= j) acc = fma(b[i * 17 + l], x[l], acc);
+            x[i] = -acc * rdiag[p + i];
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) S[(p + i) * SP + p + j] = x[i];
       }
     }
     __syncthreads();
   }
   for (int sz = 16; sz < NB; sz *= 2) {
     const int pairs = NB / (2 * sz);
-    // T = B * C^-1 for every pair (B: rows p..p+sz, cols p+sz..p+2sz of V)
+    // T = B * C^-1 for every pair (B: rows p..p+sz, cols p+sz..p+2sz, still V there)
     for (int e = tid; e < pairs * sz * sz; e += DIAG_THREADS) {
       const int pr = e / (sz * sz), r = (e / sz) % sz, cc = e % sz;
       const int p = pr * 2 * sz;
-      real acc = 0;
-      for (int l = 0; l <= cc; ++l) acc = fma(S[(p + r) * SP + p + sz + l], X[(p + sz + l) * SP + p + sz + cc], acc);
-      T[(pr * sz + r) * SP + cc] = acc;
+      const real* brow = S + (p + r) * SP + p + sz;
+      const real* ccol = S + (p + sz) * SP + p + sz + cc;
+      real a0 = 0, a1 = 0;
+      int l = 0;
+      for (; l + 1 <= cc; l += 2) {
+        a0 = fma(brow[l], ccol[l * SP], a0);
+        a1 = fma(brow[l + 1], ccol[(l + 1) * SP], a1);
+      }
+      if (l <= cc) a0 = fma(brow[l], ccol[l * SP], a0);
+      T[(pr * sz + r) * TP + cc] = a0 + a1;
     }
     __syncthreads();
-    // X12 = -A^-1 * T
+    // X12 = -A^-1 * T, written over B
     for (int e = tid; e < pairs * sz * sz; e += DIAG_THREADS) {
       const int pr = e / (sz * sz), r = (e / sz) % sz, cc = e % sz;
       const int p = pr * 2 * sz;
-      real acc = 0;
-      for (int l = r; l < sz; ++l) acc = fma(X[(p + r) * SP + p + l], T[(pr * sz + l) * SP + cc], acc);
-      X[(p + r) * SP + p + sz + cc] = -acc;
+      const real* arow = S + (p + r) * SP + p;
+      const real* tcol = T + (pr * sz) * TP + cc;
+      real a0 = 0, a1 = 0;
+      int l = r;
+      for (; l + 1 < sz; l += 2) {
+        a0 = fma(arow[l], tcol[l * TP], a0);
+        a1 = fma(arow[l + 1], tcol[(l + 1) * TP], a1);
+      }
+      if (l < sz) a0 = fma(arow[l], tcol[l * TP], a0);
+      S[(p + r) * SP + p + sz + cc] = -(a0 + a1);
     }
     __syncthreads();
   }
 
   for (int e = tid; e < nb * nb; e += DIAG_THREADS) {
     const int i = e / nb, j = e % nb;
-    if (i <= j) A[(k0 + i) * lda + k0 + j] = S[i * SP + j];
-    Winv[(k0 + i) * NB + j] = X[i * SP + j];
+    R[(k0 + i) * lda + k0 + j] = (i <= j) ? S[i * SP + j] : real(0);
   }
   if (tid == 0 && bad) atomicExch(status, kStatusNotPD);
 }
 
-__global__ void set_diag_kernel(real* R, int64_t n, real v) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i < n) R[i * n + i] = v;
+constexpr int DIAG_SMEM = (NB * SP + (NB / 2) * TP + 2 * NB + (NB / 16) * 16 * 17) * static_cast<int>(sizeof(real));
+
+
+// Recursion plan: block [lo, hi) splits at hi - n2 with n2 = ceil(n/2) rounded up to a
+// multiple of NB; blocks of at most NB are leaves.
+int64_t right_part(int64_t n) {
+  const int64_t half = (n + 1) / 2;
+  return std::min<int64_t>(n - 1, ((half + NB - 1) / NB) * NB);
 }
 
-constexpr int DIAG_SMEM = (2 * NB * SP + (NB / 2) * SP + NB) * static_cast<int>(sizeof(real));
+// Largest P (n1 x n2) over all nodes, and largest T per recursion depth.
+void plan(int64_t n, int depth, size_t& pmax, std::vector<size_t>& tmax) {
+  if (n <= NB) return;
+  const int64_t n2 = right_part(n), n1 = n - n2;
+  const size_t sz = static_cast<size_t>(n1) * n2;
+  pmax = std::max(pmax, sz);
+  if (static_cast<int>(tmax.size()) <= depth) tmax.resize(depth + 1, 0);
+  tmax[depth] = std::max(tmax[depth], sz);
+  plan(n2, depth + 1, pmax, tmax);
+  plan(n1, depth + 1, pmax, tmax);
+}
+
+struct Scratch {
+  real* P;
+  std::vector<real*> T;
+};
+
+size_t scratch_elems(int64_t n, Scratch* out, real* base) {
+  size_t pmax = 0;
+  std::vector<size_t> tmax;
+  plan(n, 0, pmax, tmax);
+  size_t off = 0;
+  auto take = [&](size_t e) {
+    real* p = base ? base + off : nullptr;
+    off += (e + 31) & ~size_t(31);
+    return p;
+  };
+  real* P = take(pmax);
+  if (out) out->P = P;
+  for (size_t d = 0; d < tmax.size(); ++d) {
+    real* t = take(tmax[d]);
+    if (out) out->T.push_back(t);
+  }
+  return off;
+}
+
+// Factor and invert the block [lo, hi) of A (upper triangle valid: the Schur complement
+// with respect to every column right of hi); writes U[lo:hi, lo:hi].
+int factor_rec(real* A, real* R, int64_t n, int64_t lo, int64_t hi, int depth, Scratch& sc, int* status,
+               cudaStream_t s) {
+  const int64_t m = hi - lo;
+  if (m <= NB) {
+    chol_diag_kernel<<<1, DIAG_THREADS, DIAG_SMEM, s>>>(A, n, lo, static_cast<int>(m), R, status);
+    return after_launch();
+  }
+  const int64_t n2 = right_part(m), n1 = m - n2, mid = hi - n2;
+  GPTQ_TRY(factor_rec(A, R, n, mid, hi, depth + 1, sc, status, s));
+  real* U22 = R + mid * n + mid;
+  real* P = sc.P;
+  real* T = sc.T[depth];
+  // P = B U22^T
+  GPTQ_TRY(dgemm(s, n1, n2, n2, 1.0, A + lo * n + mid, n, U22, n, true, 0.0, P, n2, false, kTriBTUpper));
+  // A' = A - P P^T (upper tiles)
+  GPTQ_TRY(dgemm(s, n1, n1, n2, -1.0, P, n2, P, n2, true, 1.0, A + lo * n + lo, n, true));
+  // T = P U22
+  GPTQ_TRY(dgemm(s, n1, n2, n2, 1.0, P, n2, U22, n, false, 0.0, T, n2, false, kTriBUpper));
+  GPTQ_TRY(factor_rec(A, R, n, lo, mid, depth + 1, sc, status, s));
+  // U12 = -U11 T
+  return dgemm(s, n1, n2, n1, -1.0, R + lo * n + lo, n, T, n2, false, 0.0, R + lo * n + mid, n, false, kTriAUpper);
+}
 
 }  // namespace
 
-size_t factor_small_bytes(int64_t n) {
-  return static_cast<size_t>(n) * NB * sizeof(real) + 256;
-}
+size_t factor_small_bytes(int64_t n) { return 256; }
 
-size_t factor_work_bytes(int64_t n) { return static_cast<size_t>(n) * n * sizeof(real); }
+size_t factor_work_bytes(int64_t n) {
+  return (static_cast<size_t>(n) * n + scratch_elems(n, nullptr, nullptr)) * sizeof(real);
+}
 
 int factor_hessian(const float* H, int64_t n, float damp, bool desc_act, double* U, int32_t* perm,
                    int32_t* invperm, void* work, void* small, int* status, cudaStream_t s) {
@@ -219,9 +347,9 @@ int factor_hessian(const float* H, int64_t n, float damp, bool desc_act, double*
                                                  DIAG_SMEM);
   if (attr != cudaSuccess) return GPTQ_ERR_CUDA;
   double* dsum = reinterpret_cast<double*>(small);
-  real* Winv = reinterpret_cast<real*>(static_cast<char*>(small) + 256);
-  real* A = static_cast<real*>(work);   // damped Hessian, then V
-  real* R = U;                          // V^-1, written in place into the output
+  real* A = static_cast<real*>(work);  // damped (permuted) Hessian, then Schur complements
+  Scratch sc;
+  scratch_elems(n, &sc, A + static_cast<size_t>(n) * n);
 
   GPTQ_CUDA(cudaMemsetAsync(dsum, 0, sizeof(double), s));
   diag_sum_kernel<<<std::min<int64_t>((n + 255) / 256, 148), 256, 0, s>>>(H, n, dsum);
@@ -233,38 +361,9 @@ int factor_hessian(const float* H, int64_t n, float damp, bool desc_act, double*
   const dim3 rgrid(static_cast<unsigned>((n + 255) / 256), static_cast<unsigned>(n));
   permute_damp_kernel<<<rgrid, 256, 0, s>>>(H, n, desc_act ? perm : nullptr, dsum, damp, A);
   GPTQ_TRY(after_launch());
-
-  // Reverse (bottom-right first) blocked Cholesky: A -> V (upper), H_d = V V^T.
-  const int64_t nblk = (n + NB - 1) / NB;
-  for (int64_t k = nblk - 1; k >= 0; --k) {
-    const int64_t k0 = k * NB;
-    const int nb = static_cast<int>(std::min<int64_t>(NB, n - k0));
-    chol_diag_kernel<<<1, DIAG_THREADS, DIAG_SMEM, s>>>(A, n, k0, nb, Winv, status);
-    GPTQ_TRY(after_launch());
-    if (k0 > 0) {
-      // Panel: V[0:k0, k] = A[0:k0, k] * V_kk^-T   (in place; N = nb <= 128)
-      GPTQ_TRY(dgemm(s, k0, nb, nb, 1.0, A + k0, n, Winv + k0 * NB, NB, true, 0.0, A + k0, n, false));
-      // Trailing: A[0:k0, 0:k0] -= V[0:k0, k] V[0:k0, k]^T   (upper tiles only)
-      GPTQ_TRY(dgemm(s, k0, k0, nb, -1.0, A + k0, n, A + k0, n, true, 1.0, A, n, true));
-    }
-  }
-
-  // R = V^-1 by block back substitution on the identity, bottom block row first.
-  GPTQ_CUDA(cudaMemsetAsync(R, 0, static_cast<size_t>(n) * n * sizeof(real), s));
-  set_diag_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(R, n, 1.0);
-  GPTQ_TRY(after_launch());
-  for (int64_t k = nblk - 1; k >= 0; --k) {
-    const int64_t k0 = k * NB;
-    const int nb = static_cast<int>(std::min<int64_t>(NB, n - k0));
-    // R[k, k0:] = V_kk^-1 * R[k, k0:]   (in place; M = nb <= 128)
-    GPTQ_TRY(dgemm(s, nb, n - k0, nb, 1.0, Winv + k0 * NB, NB, R + k0 * n + k0, n, false, 0.0, R + k0 * n + k0, n,
-                   false));
-    if (k0 > 0) {
-      // R[0:k0, k0:] -= V[0:k0, k] * R[k, k0:]
-      GPTQ_TRY(dgemm(s, k0, n - k0, nb, -1.0, A + k0, n, R + k0 * n + k0, n, false, 1.0, R + k0, n, false));
-    }
-  }
-  return GPTQ_OK;
+  // U starts as zeros: the GEMMs skip its (exactly zero) lower triangle.
+  GPTQ_CUDA(cudaMemsetAsync(U, 0, static_cast<size_t>(n) * n * sizeof(real), s));
+  return factor_rec(A, U, n, 0, n, 0, sc, status, s);
 }
 
 }  // namespace gptq

@@ -26,11 +26,12 @@ constexpr int64_t kNoAllocMaxN = 1024;  // largest n_in this entry point accepts
 constexpr size_t kAlign = 256;
 constexpr size_t align_up(size_t b) { return (b + kAlign - 1) & ~(kAlign - 1); }
 
-// Scratch layout for n = kNoAllocMaxN: the damped Hessian in fp64, then the small
-// factor buffers (diagonal-block inverses, diag sum), the inverse permutation and the
-// status word.
-constexpr size_t kWorkBytes = static_cast<size_t>(kNoAllocMaxN) * kNoAllocMaxN * sizeof(double);
-constexpr size_t kSmallBytes = static_cast<size_t>(kNoAllocMaxN) * 64 * sizeof(double) + 256;
+// Scratch layout for n = kNoAllocMaxN: the factor's fp64 work area (the damped Hessian
+// plus the recursion's product buffers: 1,658,880 doubles at n = 1024), the small factor
+// buffer (diag sum), the inverse permutation and the status word.  The entry point
+// re-checks at run time that the factor's needs fit.
+constexpr size_t kWorkBytes = size_t(1658880) * sizeof(double);
+constexpr size_t kSmallBytes = 256;
 constexpr size_t kPermBytes = static_cast<size_t>(kNoAllocMaxN) * sizeof(int32_t);
 constexpr size_t kScratchBytes = align_up(kWorkBytes) + align_up(kSmallBytes) + align_up(kPermBytes) + kAlign;
 

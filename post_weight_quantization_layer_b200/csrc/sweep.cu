@@ -168,8 +168,8 @@ __global__ void __launch_bounds__(256) sweep_panel_kernel(PanelArgs a) {
   extern __shared__ __align__(16) unsigned char psm[];
   double* Us = reinterpret_cast<double*>(psm);               // [PW][PW], U[j0 + r][j0 + c]
   double* rdiag = reinterpret_cast<double*>(Us + PW * PW);   // [PW], 1 / U[j][j]
-  float* ps = reinterpret_cast<float*>(rdiag + PW);          // [PW][ROWS] scale per column and row
-  int* pz = reinterpret_cast<int*>(ps + PW * ROWS);          // [PW][ROWS] zero point
+  float* ps = reinterpret_cast<float*>(rdiag + PW);          // [ROWS][PW] scale per row and column
+  int* pz = reinterpret_cast<int*>(ps + PW * ROWS);          // [ROWS][PW] zero point
   uint8_t* cs = reinterpret_cast<uint8_t*>(pz + PW * ROWS);  // [PW][ROWS] codes of this CTA
   const int tid = threadIdx.x, lane = tid & 31;
   const int tsub = tid % TPR;
@@ -195,8 +195,8 @@ __global__ void __launch_bounds__(256) sweep_panel_kernel(PanelArgs a) {
       const int64_t j = j0 + c;
       int64_t g = 0;
       if (a.gsz > 0) g = (a.static_groups && a.perm) ? clamp_idx(a.perm[j], n_in) / a.gsz : j / a.gsz;
-      ps[c * ROWS + rloc] = active ? a.scales[g * n_out + row] : 1.f;
-      pz[c * ROWS + rloc] = active ? a.zeros[g * n_out + row] : 0;
+      ps[rloc * PW + c] = active ? a.scales[g * n_out + row] : 1.f;
+      pz[rloc * PW + c] = active ? a.zeros[g * n_out + row] : 0;
     }
   }
   // The panel's running weights live in registers in fp64: each column of the panel
@@ -216,53 +216,57 @@ __global__ void __launch_bounds__(256) sweep_panel_kernel(PanelArgs a) {
   int z = 0;
   double lsum = 0.0;
 
+  // Column c = m * TPR + o is owned by the thread with tsub == o, in its register v[m].
+  // Only the loop over m is unrolled (static register indices); the loop over o stays
+  // rolled so the kernel fits the instruction cache.
 #pragma unroll
-  for (int c = 0; c < PW; ++c) {
-    if (c < pw) {
+  for (int m = 0; m < NCOL; ++m) {
+#pragma unroll 1
+    for (int o = 0; o < TPR; ++o) {
+      const int c = m * TPR + o;
+      if (c >= pw) break;
       const int64_t j = j0 + c;
-      if (a.in_panel_params) {
-        if (j % a.gsz == 0) {
-          float mn = INFINITY, mx = -INFINITY;
+      if (a.in_panel_params && j % a.gsz == 0) {
+        float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
-          for (int m = c / TPR; m < NCOL; ++m) {
-            const int col = tsub + TPR * m;
-            if (col >= c && col < c + a.gsz) {
-              const float x = static_cast<float>(v[m]);
-              mn = fminf(mn, x);
-              mx = fmaxf(mx, x);
-            }
+        for (int mm = m; mm < NCOL; ++mm) {
+          const int col = tsub + TPR * mm;
+          if (col >= c && col < c + a.gsz && col < pw) {
+            const float x = static_cast<float>(v[mm]);
+            mn = fminf(mn, x);
+            mx = fmaxf(mx, x);
           }
+        }
 #pragma unroll
-          for (int off = 1; off < TPR; off <<= 1) {
-            mn = fminf(mn, __shfl_xor_sync(FULL, mn, off));
-            mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, off));
-          }
-          group_params(mn, mx, a.bits, a.sym != 0, s, z);
-          if (tsub == 0 && active) {
-            a.scales[(j / a.gsz) * n_out + row] = s;
-            a.zeros[(j / a.gsz) * n_out + row] = z;
-          }
+        for (int off = 1; off < TPR; off <<= 1) {
+          mn = fminf(mn, __shfl_xor_sync(FULL, mn, off));
+          mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, off));
+        }
+        group_params(mn, mx, a.bits, a.sym != 0, s, z);
+        if (tsub == 0 && active) {
+          a.scales[(j / a.gsz) * n_out + row] = s;
+          a.zeros[(j / a.gsz) * n_out + row] = z;
         }
       }
       double err = 0.0;
-      if (tsub == (c % TPR)) {
+      if (tsub == o) {
         if (!a.in_panel_params) {
-          s = ps[c * ROWS + rloc];
-          z = pz[c * ROWS + rloc];
+          s = ps[rloc * PW + c];
+          z = pz[rloc * PW + c];
         }
-        const double w = v[c / TPR];
+        const double w = v[m];
         const int q = quant_code(static_cast<float>(w), s, z, maxq);
         const double what = static_cast<double>(s) * static_cast<double>(q - z);
         err = (w - what) * rdiag[c];
-        v[c / TPR] = err;
+        v[m] = err;
         cs[c * ROWS + rloc] = static_cast<uint8_t>(q);
         lsum += err * err;
       }
-      err = __shfl_sync(FULL, err, base_lane + (c % TPR));
+      err = __shfl_sync(FULL, err, base_lane + o);
 #pragma unroll
-      for (int m = c / TPR; m < NCOL; ++m) {
-        const int col = tsub + TPR * m;
-        if (col > c) v[m] = fma(-err, Us[c * PW + col], v[m]);
+      for (int mm = m; mm < NCOL; ++mm) {
+        const int col = tsub + TPR * mm;
+        if (col > c) v[mm] = fma(-err, Us[c * PW + col], v[mm]);
       }
     }
   }
