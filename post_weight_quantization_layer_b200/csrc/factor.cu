@@ -114,13 +114,16 @@ __global__ void __launch_bounds__(DIAG_THREADS) chol_diag_kernel(const real* A, 
   real* rdiag = col + NB;               // [NB] 1 / V[j][j]
   real* blk = rdiag + NB;               // [NB/16][16][17] copies of the 16x16 diagonal blocks
   __shared__ int bad;
-  __shared__ real colbuf[2][NB];        // column c of the running matrix, double-buffered
+  // Column c of the running matrix (+ 1/pivot), double-buffered; row i lives at q(i) =
+  // i + i/4 so that the 32 lanes of a warp (4 rows each) read it without bank conflicts.
+  constexpr int QN = NB + NB / 4 + 1;
+  __shared__ real colbuf[2][QN];
   const int tid = threadIdx.x;
   if (tid == 0) bad = 0;
-  // Register blocking: thread (rb, cb) holds rows 4rb..4rb+3 x cols 8cb..8cb+7 of the block
-  // (upper triangle; the identity pads it to NB x NB).
-  const int rb = tid >> 4, cb = tid & 15;
-  const int i0 = rb * 4, j0 = cb * 8;
+  // Register blocking: warp w holds columns 8w..8w+7 and lane l rows 4l..4l+3 of the block,
+  // so a column is owned by one whole warp and column reads are warp-uniform broadcasts.
+  const int lane = tid & 31, wcol = tid >> 5;
+  const int i0 = lane * 4, j0 = wcol * 8;
   real r[4][8];
 #pragma unroll
   for (int a = 0; a < 4; ++a)
@@ -136,57 +139,74 @@ __global__ void __launch_bounds__(DIAG_THREADS) chol_diag_kernel(const real* A, 
       }
       r[a][b] = v;
     }
+  __syncthreads();  // `bad` is initialised before any owner may set it
   // Reverse Cholesky: for c = NB-1 .. 0, V[c][c] = sqrt(S[c][c]), V[i][c] = S[i][c] / V[c][c]
-  // for i < c, then S[i][j] -= V[i][c] V[j][c] for i <= j < c.
+  // for i < c, then S[i][j] -= V[i][c] V[j][c] for j < c.  Elements below the diagonal are
+  // updated too (their values are never read and are zeroed at the end), which keeps every
+  // branch warp-uniform.
   for (int c = NB - 1; c >= 0; --c) {
-    real* cb_buf = colbuf[c & 1];
-    if (cb == (c >> 3)) {
+    real* buf = colbuf[c & 1];
+    if (wcol == (c >> 3)) {  // the owner warp publishes column c
+      const int bc = c & 7;
 #pragma unroll
       for (int b = 0; b < 8; ++b)
-        if (j0 + b == c) {
-#pragma unroll
-          for (int a = 0; a < 4; ++a)
-            if (i0 + a <= c) cb_buf[i0 + a] = r[a][b];
-        }
-    }
-    __syncthreads();
-    real d = cb_buf[c];
-    if (!(d > 0) || !isfinite(d)) {
-      if (tid == 0) bad = 1;
-      d = 1;
-    }
-    const real v = sqrt(d);
-    const real rv = 1 / v;
-    if (j0 < c && i0 < c) {
-      real ci[4], cj[8];
-#pragma unroll
-      for (int a = 0; a < 4; ++a) ci[a] = cb_buf[min(i0 + a, c)] * rv;
-#pragma unroll
-      for (int b = 0; b < 8; ++b) cj[b] = cb_buf[min(j0 + b, c)] * rv;
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 8; ++b)
-          if (i0 + a <= j0 + b && j0 + b < c) r[a][b] = fma(-ci[a], cj[b], r[a][b]);
-    }
-    if (cb == (c >> 3)) {  // finish column c of V in registers
-#pragma unroll
-      for (int b = 0; b < 8; ++b)
-        if (j0 + b == c) {
+        if (b == bc) {
 #pragma unroll
           for (int a = 0; a < 4; ++a) {
-            if (i0 + a < c) r[a][b] *= rv;
-            if (i0 + a == c) r[a][b] = v;
+            const int i = i0 + a;
+            if (i <= c) buf[i + (i >> 2)] = r[a][b];
+            if (i == c) {
+              real d = r[a][b];
+              if (!(d > 0) || !isfinite(d)) {
+                bad = 1;
+                d = 1;
+              }
+              const real v = sqrt(d);
+              r[a][b] = v;
+              buf[QN - 1] = 1 / v;
+              rdiag[c] = 1 / v;
+            }
           }
         }
     }
-    if (tid == 0) rdiag[c] = rv;
+    __syncthreads();
+    const real rv = buf[QN - 1];
+    if (j0 < c) {
+      real ci[4], cj[8];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) ci[a] = buf[(i0 + a) + ((i0 + a) >> 2)] * rv;
+#pragma unroll
+      for (int b = 0; b < 8; ++b) cj[b] = buf[min(j0 + b, c) + (min(j0 + b, c) >> 2)] * rv;
+      if (j0 + 7 < c) {
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int b = 0; b < 8; ++b) r[a][b] = fma(-ci[a], cj[b], r[a][b]);
+      } else {  // the warp that holds column c: only its columns j < c
+#pragma unroll
+        for (int b = 0; b < 8; ++b)
+          if (j0 + b < c) {
+#pragma unroll
+            for (int a = 0; a < 4; ++a) r[a][b] = fma(-ci[a], cj[b], r[a][b]);
+          }
+      }
+    }
+    if (wcol == (c >> 3)) {  // finish column c of V in registers
+      const int bc = c & 7;
+#pragma unroll
+      for (int b = 0; b < 8; ++b)
+        if (b == bc) {
+#pragma unroll
+          for (int a = 0; a < 4; ++a)
+            if (i0 + a < c) r[a][b] *= rv;
+        }
+    }
   }
-  // V to shared memory for the inverse
+  // V to shared memory for the inverse (zero below the diagonal)
 #pragma unroll
   for (int a = 0; a < 4; ++a)
 #pragma unroll
-    for (int b = 0; b < 8; ++b) S[(i0 + a) * SP + j0 + b] = r[a][b];
+    for (int b = 0; b < 8; ++b) S[(i0 + a) * SP + j0 + b] = (i0 + a <= j0 + b) ? r[a][b] : real(0);
   __syncthreads();
 
   // V^-1 in place by doubling: invert the 16x16 diagonal blocks, then join neighbours with
