@@ -21,9 +21,10 @@
 //   long chain of rounding decisions, each depending on every earlier error of its row,
 //   so fp32-level perturbations of the running weights grow into different codes over
 //   thousands of columns.
-// * Two-level lazy updates: after each panel its errors update the rest of the current
-//   outer block (<= 1024 columns); after each outer block its errors update every later
-//   column in one GEMM with K = outer block width.
+// * Two-level lazy updates: inside an outer block (<= 512 columns) each panel kernel first
+//   applies the pending errors of the block's earlier panels to its own columns (a small
+//   left-looking product on the fp64 matrix units); after each outer block its errors
+//   update every later column in one GEMM with K = outer block width.
 #include <algorithm>
 
 #include "common.cuh"
@@ -37,7 +38,16 @@ constexpr int NCOL = PW / TPR;         // columns per thread
 constexpr int ROWS = 256 / TPR;        // rows per CTA
 // U block (fp64) + per-column reciprocal pivots (fp64) + per-column group parameters of
 // every row (scale fp32, zero int32) + codes.
-constexpr int PANEL_SMEM = PW * PW * 8 + PW * 8 + PW * ROWS * 8 + PW * ROWS;
+constexpr int KC = 32;                 // K chunk of the fused left-looking update
+constexpr int EP = KC + 4, UP = PW + 4;  // padded pitches (conflict-free fragment loads)
+constexpr int PANEL_SMEM = PW * PW * 8 + PW * 8 + PW * ROWS * 8 + PW * ROWS +
+                           (2 * (ROWS * EP + KC * UP) + ROWS * UP) * 8;
+constexpr int OUTER = 512;             // outer block width (left-looking K stays below it)
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool pred) {
+  const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(sa), "l"(gmem), "r"(pred ? 16 : 0) : "memory");
+}
 
 // ---------------------------------------------------------------- quantizer (float32 decisions)
 __device__ __forceinline__ void params_sym(float amax, int bits, float& s, int& z) {
@@ -152,6 +162,7 @@ struct PanelArgs {
   int64_t n_out, n_in;
   const double* U;
   int64_t j0;
+  int64_t o0;  // first column of the current outer block (errors of [o0, j0) are still pending)
   int pw;
   int bits, gsz;
   int sym;
@@ -171,6 +182,9 @@ __global__ void __launch_bounds__(256) sweep_panel_kernel(PanelArgs a) {
   float* ps = reinterpret_cast<float*>(rdiag + PW);          // [ROWS][PW] scale per row and column
   int* pz = reinterpret_cast<int*>(ps + PW * ROWS);          // [ROWS][PW] zero point
   uint8_t* cs = reinterpret_cast<uint8_t*>(pz + PW * ROWS);  // [PW][ROWS] codes of this CTA
+  double* Es = reinterpret_cast<double*>(cs + PW * ROWS);    // [2][ROWS][EP] chunks of Err
+  double* Ut = Es + 2 * ROWS * EP;                            // [2][KC][UP] chunks of U rows
+  double* Cs = Ut + 2 * KC * UP;                              // [ROWS][UP] accumulated update
   const int tid = threadIdx.x, lane = tid & 31;
   const int tsub = tid % TPR;
   const int rloc = tid / TPR;
@@ -210,6 +224,85 @@ __global__ void __launch_bounds__(256) sweep_panel_kernel(PanelArgs a) {
   }
   __syncthreads();
   if (tid < pw) rdiag[tid] = 1.0 / Us[tid * PW + tid];
+
+  // Left-looking part of the lazy update: the errors of the earlier panels of this outer
+  // block, Err[rows, o0:j0] U[o0:j0, panel], are applied here instead of by a separate
+  // GEMM per panel.  fp64 on the fp64 matrix units: warp w computes columns 8w..8w+7 of
+  // the 16 x 64 product as two m8n8 tiles.
+  if (a.j0 > a.o0) {
+    const int g = lane >> 2, t = lane & 3, w = tid >> 5;
+    double acc[2][2] = {{0.0, 0.0}, {0.0, 0.0}};
+    const int nch = static_cast<int>((j0 - a.o0 + KC - 1) / KC);
+    // Chunk ch covers error columns [o0 + ch*KC, ...); both tiles are fetched with
+    // 16-byte cp.async (zero-filled outside the matrix), two chunks in flight.
+    // 16-byte copies need even element offsets; odd panel widths (odd group sizes) take
+    // the plain-load path.
+    const bool vec_ok = ((j0 | a.o0 | n_in | static_cast<int64_t>(pw)) & 1) == 0;
+    auto stage = [&](int ch, int buf) {
+      const int64_t k0 = a.o0 + static_cast<int64_t>(ch) * KC;
+      if (!vec_ok) {
+        for (int e = tid; e < ROWS * KC; e += 256) {
+          const int r = e / KC, k = e % KC;
+          const int64_t gr = row0 + r, gk = k0 + k;
+          Es[buf * ROWS * EP + r * EP + k] = (gr < n_out && gk < j0) ? a.Err[gr * n_in + gk] : 0.0;
+        }
+        for (int e = tid; e < KC * PW; e += 256) {
+          const int k = e / PW, c = e % PW;
+          const int64_t gk = k0 + k;
+          Ut[buf * KC * UP + k * UP + c] = (gk < j0 && c < pw) ? a.U[gk * n_in + j0 + c] : 0.0;
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        return;
+      }
+      {
+        const int r = tid >> 4, kc = (tid & 15) * 2;  // 16 rows x 16 chunks
+        const int64_t gr = row0 + r, gk = k0 + kc;
+        const bool ok = gr < n_out && gk < j0;
+        cp_async16(Es + buf * ROWS * EP + r * EP + kc, ok ? a.Err + gr * n_in + gk : a.Err, ok);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {                   // 32 rows x 32 chunks
+        const int e = tid + 256 * i;
+        const int k = e >> 5, c = (e & 31) * 2;
+        const int64_t gk = k0 + k;
+        const bool ok = gk < j0 && c < pw;
+        cp_async16(Ut + buf * KC * UP + k * UP + c, ok ? a.U + gk * n_in + j0 + c : a.U, ok);
+      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    stage(0, 0);
+    for (int ch = 0; ch < nch; ++ch) {
+      if (ch + 1 < nch) {
+        stage(ch + 1, (ch + 1) & 1);
+        asm volatile("cp.async.wait_group 1;" ::: "memory");
+      } else {
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+      }
+      __syncthreads();
+      const double* es = Es + (ch & 1) * ROWS * EP;
+      const double* ut = Ut + (ch & 1) * KC * UP;
+#pragma unroll
+      for (int kk = 0; kk < KC; kk += 4) {
+        const double b0 = ut[(kk + t) * UP + w * 8 + g];
+#pragma unroll
+        for (int mb = 0; mb < 2; ++mb) {
+          const double a0 = es[(mb * 8 + g) * EP + kk + t];
+          asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+                       : "+d"(acc[mb][0]), "+d"(acc[mb][1])
+                       : "d"(a0), "d"(b0));
+        }
+      }
+      __syncthreads();
+    }
+#pragma unroll
+    for (int mb = 0; mb < 2; ++mb) {
+      Cs[(mb * 8 + g) * UP + w * 8 + 2 * t] = acc[mb][0];
+      Cs[(mb * 8 + g) * UP + w * 8 + 2 * t + 1] = acc[mb][1];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < NCOL; ++m) v[m] -= Cs[rloc * UP + tsub + TPR * m];
+  }
   __syncthreads();
 
   float s = 1.f;
@@ -393,9 +486,12 @@ int run_sweep(SweepArgs& a, cudaStream_t s, int* panel_width, int* outer_width) 
         }
     }
   }
-  // Outer block: a multiple of P (and of g when groups are wider than a panel).
-  int64_t base = (dynamic_groups && g > P) ? g : P;
-  int64_t Q = base * std::max<int64_t>(1, 1024 / base);
+  // Outer block: a multiple of P.  When groups wider than a panel take their parameters
+  // from the current weights, the outer block is the group itself, so that every earlier
+  // error has reached the whole group (through the outer update) when its parameters are
+  // computed at its first column.
+  const int64_t Q = (dynamic_groups && g > P) ? static_cast<int64_t>(g)
+                                              : static_cast<int64_t>(P) * std::max<int64_t>(1, OUTER / P);
   if (panel_width) *panel_width = P;
   if (outer_width) *outer_width = static_cast<int>(std::min<int64_t>(Q, n_in));
 
@@ -436,13 +532,11 @@ int run_sweep(SweepArgs& a, cudaStream_t s, int* panel_width, int* outer_width) 
         GPTQ_TRY(after_launch());
       }
       pa.j0 = p0;
+      pa.o0 = O0;
       pa.pw = static_cast<int>(p1 - p0);
       pa.in_panel_params = (dynamic_groups && g <= P) ? 1 : 0;
       sweep_panel_kernel<<<panel_grid, 256, PANEL_SMEM, s>>>(pa);
       GPTQ_TRY(after_launch());
-      if (p1 < O1)  // rest of the outer block: W[:, p1:O1] -= Err[:, p0:p1] U[p0:p1, p1:O1]
-        GPTQ_TRY(dgemm(s, n_out, O1 - p1, p1 - p0, -1.0, a.Err + p0, n_in, a.U + p0 * n_in + p1, n_in, false, 1.0,
-                       a.Wk + p1, n_in, false));
     }
     if (O1 < n_in)  // every later column: W[:, O1:] -= Err[:, O0:O1] U[O0:O1, O1:]
       GPTQ_TRY(dgemm(s, n_out, n_in - O1, O1 - O0, -1.0, a.Err + O0, n_in, a.U + O0 * n_in + O1, n_in, false, 1.0,

@@ -135,3 +135,11 @@ def test_trim_workspace_keeps_library_usable():
     assert _native.lib().gptq_trim_workspace() == 0
     b = gq.quantize_layer(W.to(dev), H.to(dev), 4, 32)
     assert torch.equal(a.qweight, b.qweight)
+
+
+@pytest.mark.parametrize("n_out,n_in,g", [(20, 48, 3), (33, 120, 15), (17, 200, 25)])
+def test_odd_group_sizes(n_out, n_in, g):
+    """Odd group sizes make odd panel widths (63, 60, 50 columns) and odd panel starts."""
+    W, H = _problem(n_out, n_in, 8 * n_in, n_in + g, w_dtype=torch.float32)
+    _, _, m = _run(W, H, 4, g, False, False, False)
+    assert_parity(m, (n_out, n_in, g))
