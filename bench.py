@@ -241,7 +241,7 @@ def run_native(args, world, rank, local):
     per_launch = [work["hessian_flops"][i] / (launch_ms[i] / 1e3) / 1e12 for i in range(len(launch_ms))]
     f_tflops = sum(work["factor_flops"]) / (f_ms / 1e3) / 1e12
     s_tflops = sum(work["sweep_flops"]) / (s_ms / 1e3) / 1e12
-    fp32_simt_peak = props.multi_processor_count * 128 * 2 * peaks["sm_max"] * 1e6 / 1e12
+    fp64_peak = measure_fp64_peak(dev)
 
     roofline = {
         "kernel": "hessian_syrk_kernel (tcgen05 kind::f16, bf16 in, fp32 accumulate)",
@@ -262,13 +262,14 @@ def run_native(args, world, rank, local):
     phases = {
         "hessian": {"ms": round(h_ms, 3), "tflops": round(h_tflops, 1),
                     "frac_of_bf16_sustained": round(h_tflops / peaks["bf16_sus"], 4)},
-        "factor": {"ms": round(f_ms, 3), "tflops": round(f_tflops, 2),
-                   "frac_of_fp32_simt_peak": round(f_tflops / fp32_simt_peak, 4),
-                   "fp32_simt_peak_tflops": round(fp32_simt_peak, 1)},
-        "sweep": {"ms": round(s_ms, 3), "tflops": round(s_tflops, 2),
-                  "frac_of_fp32_simt_peak": round(s_tflops / fp32_simt_peak, 4),
+        "factor": {"ms": round(f_ms, 3), "tflops_fp64": round(f_tflops, 2),
+                   "frac_of_fp64_peak": round(f_tflops / fp64_peak, 4)},
+        "sweep": {"ms": round(s_ms, 3), "tflops_fp64": round(s_tflops, 2),
+                  "frac_of_fp64_peak": round(s_tflops / fp64_peak, 4),
                   "min_hbm_gbs": round(work["sweep_min_bytes"] / (s_ms / 1e3) / 1e9, 1),
                   "frac_of_hbm": round(work["sweep_min_bytes"] / (s_ms / 1e3) / 1e9 / peaks["hbm"], 4)},
+        "fp64_peak_tflops": round(fp64_peak, 1),
+        "fp64_peak_how": "measured in this run: cuBLAS fp64 GEMM 8192^3 (torch.matmul), best of 3",
     }
 
     e2e = None
@@ -300,6 +301,26 @@ def run_native(args, world, rank, local):
         "cpu_baseline": cpu,
     }
     return line
+
+
+def measure_fp64_peak(dev):
+    """Denominator of the fp64 phases: this GPU's fp64 GEMM rate, measured with cuBLAS."""
+    import torch
+    n = 8192
+    a = torch.randn(n, n, device=dev, dtype=torch.float64)
+    b = torch.randn(n, n, device=dev, dtype=torch.float64)
+    a @ b
+    torch.cuda.synchronize()
+    best = 1e30
+    for _ in range(3):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        a @ b
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    del a, b
+    return 2 * n ** 3 / (best / 1e3) / 1e12
 
 
 def load_traffic():
