@@ -37,8 +37,8 @@ namespace {
 
 constexpr int NB = 128;  // leaf block width of the factorisation
 constexpr int DIAG_THREADS = 512;
-constexpr int SP = NB + 1;  // padded pitch of the diagonal block in shared memory
-constexpr int TP = NB / 2 + 1;
+constexpr int SP = NB + 4;      // pitch of the diagonal block in shared memory (fragment loads
+constexpr int TP = NB / 2 + 4;  // of m8n8k4 hit 16 distinct bank pairs when pitch = 4 mod 16)
 using real = double;     // working precision of the factorisation
 
 // Sum of diag(H) in double.
@@ -95,6 +95,33 @@ __global__ void permute_damp_kernel(const float* __restrict__ H, int64_t n, cons
   A[i * n + j] = v;
 }
 
+// D = sign * A * B for shared-memory blocks (M, N multiples of 8, K of 4), all warps of the
+// CTA sharing the m8n8 output tiles, on the fp64 matrix units.  tri & 1: A is upper
+// triangular (A[m][k] == 0 for k < m); tri & 2: B is upper triangular (B[k][n] == 0 for
+// k > n); those K ranges hold exact zeros and are skipped.
+__device__ __forceinline__ void cta_dmma(real* D, int ldd, const real* A, int lda, const real* B, int ldb, int M, int N,
+                                         int K, int tri, real sign) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int tn = N / 8;
+  for (int tt = warp; tt < (M / 8) * tn; tt += DIAG_THREADS / 32) {
+    const int m0 = (tt / tn) * 8, n0 = (tt % tn) * 8;
+    int kb = 0, ke = K;
+    if (tri & 1) kb = m0;
+    if (tri & 2) ke = min(K, n0 + 8);
+    kb &= ~3;
+    real c0 = 0, c1 = 0;
+    for (int k = kb; k < ke; k += 4) {
+      const real a0 = A[(m0 + g) * lda + k + t];
+      const real b0 = B[(k + t) * ldb + n0 + g];
+      asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+                   : "+d"(c0), "+d"(c1)
+                   : "d"(a0), "d"(b0));
+    }
+    D[(m0 + g) * ldd + n0 + 2 * t] = sign * c0;
+    D[(m0 + g) * ldd + n0 + 2 * t + 1] = sign * c1;
+  }
+}
+
 // Factor the diagonal block A[k0:k0+nb, k0:k0+nb] (upper part valid) as V V^T with V upper
 // and write its inverse into R[k0:k0+nb, k0:k0+nb] (same leading dimension, zeros below the
 // diagonal).  A pivot that is not positive and finite sets *status = NOT_PD; the
@@ -114,16 +141,17 @@ __global__ void __launch_bounds__(DIAG_THREADS) chol_diag_kernel(const real* A, 
   real* rdiag = col + NB;               // [NB] 1 / V[j][j]
   real* blk = rdiag + NB;               // [NB/16][16][17] copies of the 16x16 diagonal blocks
   __shared__ int bad;
-  // Column c of the running matrix (+ 1/pivot), double-buffered; row i lives at q(i) =
-  // i + i/4 so that the 32 lanes of a warp (4 rows each) read it without bank conflicts.
-  constexpr int QN = NB + NB / 4 + 1;
-  __shared__ real colbuf[2][QN];
+  // Published 8-column panels of V, double-buffered; row i of a panel column lives at
+  // q(i) = i + i/4 so that the 32 lanes of a warp (4 rows each) read it without bank
+  // conflicts.
+  constexpr int QN = NB + NB / 4;
+  __shared__ real pbuf[2][8][QN];
   const int tid = threadIdx.x;
   if (tid == 0) bad = 0;
-  // Register blocking: warp w holds columns 8w..8w+7 and lane l rows 4l..4l+3 of the block,
-  // so a column is owned by one whole warp and column reads are warp-uniform broadcasts.
+  // Register blocking: warp w holds columns 8w..8w+7 and lane l rows 4l..4l+3 of the block.
   const int lane = tid & 31, wcol = tid >> 5;
   const int i0 = lane * 4, j0 = wcol * 8;
+  const unsigned FULLM = 0xffffffffu;
   real r[4][8];
 #pragma unroll
   for (int a = 0; a < 4; ++a)
@@ -140,66 +168,60 @@ __global__ void __launch_bounds__(DIAG_THREADS) chol_diag_kernel(const real* A, 
       r[a][b] = v;
     }
   __syncthreads();  // `bad` is initialised before any owner may set it
-  // Reverse Cholesky: for c = NB-1 .. 0, V[c][c] = sqrt(S[c][c]), V[i][c] = S[i][c] / V[c][c]
-  // for i < c, then S[i][j] -= V[i][c] V[j][c] for j < c.  Elements below the diagonal are
-  // updated too (their values are never read and are zeroed at the end), which keeps every
-  // branch warp-uniform.
-  for (int c = NB - 1; c >= 0; --c) {
-    real* buf = colbuf[c & 1];
-    if (wcol == (c >> 3)) {  // the owner warp publishes column c
-      const int bc = c & 7;
+  // Blocked reverse Cholesky over 8-column panels, right to left.  The warp owning panel p
+  // factors it alone with warp shuffles (column c: V[c][c] = sqrt(S[c][c]),
+  // V[i][c] = S[i][c] / V[c][c], then the panel's earlier columns get the rank-1 update),
+  // publishes it, and every warp holding earlier columns applies the rank-8 update
+  // S[i][j] -= sum_k V[i][8p+k] V[j][8p+k].  One barrier per panel; while the next owner
+  // factors, the other warps are still applying the previous update.  Elements below the
+  // diagonal are updated too (never read, zeroed at the end).
+  for (int p = NB / 8 - 1; p >= 0; --p) {
+    real(*pb)[QN] = pbuf[p & 1];
+    if (wcol == p) {
+#pragma unroll
+      for (int bc = 7; bc >= 0; --bc) {
+        const int c = 8 * p + bc;
+        const int src = 2 * p + (bc >> 2);  // lane holding row c (and row 8p+b for b>>2 == bc>>2)
+        real d = __shfl_sync(FULLM, r[bc & 3][bc], src);
+        if (!(d > 0) || !isfinite(d)) {
+          if (lane == src) bad = 1;
+          d = 1;
+        }
+        const real v = sqrt(d);
+        const real rv = 1 / v;
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          const int i = i0 + a;
+          if (i < c) r[a][bc] *= rv;
+          if (i == c) r[a][bc] = v;
+        }
+        if (lane == src) rdiag[c] = rv;
+#pragma unroll
+        for (int b = 0; b < bc; ++b) {
+          const real vb = __shfl_sync(FULLM, r[b & 3][bc], 2 * p + (b >> 2));  // V[8p+b][c]
+#pragma unroll
+          for (int a = 0; a < 4; ++a) r[a][b] = fma(-r[a][bc], vb, r[a][b]);
+        }
+      }
 #pragma unroll
       for (int b = 0; b < 8; ++b)
-        if (b == bc) {
 #pragma unroll
-          for (int a = 0; a < 4; ++a) {
-            const int i = i0 + a;
-            if (i <= c) buf[i + (i >> 2)] = r[a][b];
-            if (i == c) {
-              real d = r[a][b];
-              if (!(d > 0) || !isfinite(d)) {
-                bad = 1;
-                d = 1;
-              }
-              const real v = sqrt(d);
-              r[a][b] = v;
-              buf[QN - 1] = 1 / v;
-              rdiag[c] = 1 / v;
-            }
-          }
-        }
+        for (int a = 0; a < 4; ++a) pb[b][(i0 + a) + lane] = r[a][b];  // q(i0+a) = i0 + a + lane
     }
     __syncthreads();
-    const real rv = buf[QN - 1];
-    if (j0 < c) {
-      real ci[4], cj[8];
+    if (wcol < p) {
 #pragma unroll
-      for (int a = 0; a < 4; ++a) ci[a] = buf[(i0 + a) + ((i0 + a) >> 2)] * rv;
+      for (int k = 0; k < 8; ++k) {
+        real vi[4], vj[8];
 #pragma unroll
-      for (int b = 0; b < 8; ++b) cj[b] = buf[min(j0 + b, c) + (min(j0 + b, c) >> 2)] * rv;
-      if (j0 + 7 < c) {
+        for (int a = 0; a < 4; ++a) vi[a] = pb[k][(i0 + a) + lane];
+#pragma unroll
+        for (int b = 0; b < 8; ++b) vj[b] = pb[k][(j0 + b) + ((j0 + b) >> 2)];
 #pragma unroll
         for (int a = 0; a < 4; ++a)
 #pragma unroll
-          for (int b = 0; b < 8; ++b) r[a][b] = fma(-ci[a], cj[b], r[a][b]);
-      } else {  // the warp that holds column c: only its columns j < c
-#pragma unroll
-        for (int b = 0; b < 8; ++b)
-          if (j0 + b < c) {
-#pragma unroll
-            for (int a = 0; a < 4; ++a) r[a][b] = fma(-ci[a], cj[b], r[a][b]);
-          }
+          for (int b = 0; b < 8; ++b) r[a][b] = fma(-vi[a], vj[b], r[a][b]);
       }
-    }
-    if (wcol == (c >> 3)) {  // finish column c of V in registers
-      const int bc = c & 7;
-#pragma unroll
-      for (int b = 0; b < 8; ++b)
-        if (b == bc) {
-#pragma unroll
-          for (int a = 0; a < 4; ++a)
-            if (i0 + a < c) r[a][b] *= rv;
-        }
     }
   }
   // V to shared memory for the inverse (zero below the diagonal)
@@ -242,35 +264,15 @@ __global__ void __launch_bounds__(DIAG_THREADS) chol_diag_kernel(const real* A, 
   for (int sz = 16; sz < NB; sz *= 2) {
     const int pairs = NB / (2 * sz);
     // T = B * C^-1 for every pair (B: rows p..p+sz, cols p+sz..p+2sz, still V there)
-    for (int e = tid; e < pairs * sz * sz; e += DIAG_THREADS) {
-      const int pr = e / (sz * sz), r = (e / sz) % sz, cc = e % sz;
+    for (int pr = 0; pr < pairs; ++pr) {
       const int p = pr * 2 * sz;
-      const real* brow = S + (p + r) * SP + p + sz;
-      const real* ccol = S + (p + sz) * SP + p + sz + cc;
-      real a0 = 0, a1 = 0;
-      int l = 0;
-      for (; l + 1 <= cc; l += 2) {
-        a0 = fma(brow[l], ccol[l * SP], a0);
-        a1 = fma(brow[l + 1], ccol[(l + 1) * SP], a1);
-      }
-      if (l <= cc) a0 = fma(brow[l], ccol[l * SP], a0);
-      T[(pr * sz + r) * TP + cc] = a0 + a1;
+      cta_dmma(T + pr * sz * TP, TP, S + p * SP + p + sz, SP, S + (p + sz) * SP + p + sz, SP, sz, sz, sz, 2, 1);
     }
     __syncthreads();
     // X12 = -A^-1 * T, written over B
-    for (int e = tid; e < pairs * sz * sz; e += DIAG_THREADS) {
-      const int pr = e / (sz * sz), r = (e / sz) % sz, cc = e % sz;
+    for (int pr = 0; pr < pairs; ++pr) {
       const int p = pr * 2 * sz;
-      const real* arow = S + (p + r) * SP + p;
-      const real* tcol = T + (pr * sz) * TP + cc;
-      real a0 = 0, a1 = 0;
-      int l = r;
-      for (; l + 1 < sz; l += 2) {
-        a0 = fma(arow[l], tcol[l * TP], a0);
-        a1 = fma(arow[l + 1], tcol[(l + 1) * TP], a1);
-      }
-      if (l < sz) a0 = fma(arow[l], tcol[l * TP], a0);
-      S[(p + r) * SP + p + sz + cc] = -(a0 + a1);
+      cta_dmma(S + p * SP + p + sz, SP, S + p * SP + p, SP, T + pr * sz * TP, TP, sz, sz, sz, 1, -1);
     }
     __syncthreads();
   }

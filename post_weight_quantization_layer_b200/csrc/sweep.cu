@@ -13,9 +13,9 @@
 //   quantized its slot holds err_j, so the lazy updates read the errors in place.
 // * codesT [n_in, n_out] uint8 holds the codes in sweep order (column-major w.r.t. W),
 //   so both the sweep's writes and the packer's reads are coalesced across rows.
-// * Panels of P <= 64 columns: one kernel per panel, rows in parallel (16 threads per
-//   row, 4 columns per thread in registers, the panel's block of U in shared memory,
-//   group min/max and the error broadcast via warp shuffles).
+// * Panels of P <= 64 columns: one kernel per panel, rows in parallel (4 threads per row,
+//   16 columns per thread in registers, the panel's block of U in shared memory, group
+//   min/max and the error broadcast via warp shuffles).
 // * Precision: the running weights, the errors, U and the lazy-update products are all
 //   fp64; only the code decision (w / s, rounding) is taken in fp32.  GPTQ's sweep is a
 //   long chain of rounding decisions, each depending on every earlier error of its row,
@@ -33,15 +33,17 @@ namespace gptq {
 namespace {
 
 constexpr int PW = 64;                 // max panel width
-constexpr int TPR = 16;                // threads per row
+constexpr int PTHREADS = 128;          // threads per CTA of the panel kernel
+constexpr int TPR = 4;                 // threads per row
 constexpr int NCOL = PW / TPR;         // columns per thread
-constexpr int ROWS = 256 / TPR;        // rows per CTA
+constexpr int ROWS = PTHREADS / TPR;   // rows per CTA
 // U block (fp64) + per-column reciprocal pivots (fp64) + per-column group parameters of
 // every row (scale fp32, zero int32) + codes.
 constexpr int KC = 32;                 // K chunk of the fused left-looking update
 constexpr int EP = KC + 4, UP = PW + 4;  // padded pitches (conflict-free fragment loads)
-constexpr int PANEL_SMEM = PW * PW * 8 + PW * 8 + PW * ROWS * 8 + PW * ROWS +
-                           (2 * (ROWS * EP + KC * UP) + ROWS * UP) * 8;
+// (the accumulated update [ROWS][UP] reuses the U staging buffers)
+constexpr int PANEL_SMEM = PW * PW * 8 + PW * 8 + PW * ROWS * 8 + PW * ROWS + (2 * (ROWS * EP + KC * UP)) * 8;
+static_assert(ROWS * UP <= 2 * KC * UP, "accumulator tile must fit in the staging buffers");
 constexpr int OUTER = 512;             // outer block width (left-looking K stays below it)
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool pred) {
@@ -175,16 +177,16 @@ struct PanelArgs {
   double* loss;
 };
 
-__global__ void __launch_bounds__(256) sweep_panel_kernel(PanelArgs a) {
+__global__ void __launch_bounds__(PTHREADS) sweep_panel_kernel(PanelArgs a) {
   extern __shared__ __align__(16) unsigned char psm[];
   double* Us = reinterpret_cast<double*>(psm);               // [PW][PW], U[j0 + r][j0 + c]
   double* rdiag = reinterpret_cast<double*>(Us + PW * PW);   // [PW], 1 / U[j][j]
-  float* ps = reinterpret_cast<float*>(rdiag + PW);          // [ROWS][PW] scale per row and column
-  int* pz = reinterpret_cast<int*>(ps + PW * ROWS);          // [ROWS][PW] zero point
+  float* ps = reinterpret_cast<float*>(rdiag + PW);          // [PW][ROWS] scale per column and row
+  int* pz = reinterpret_cast<int*>(ps + PW * ROWS);          // [PW][ROWS] zero point
   uint8_t* cs = reinterpret_cast<uint8_t*>(pz + PW * ROWS);  // [PW][ROWS] codes of this CTA
   double* Es = reinterpret_cast<double*>(cs + PW * ROWS);    // [2][ROWS][EP] chunks of Err
   double* Ut = Es + 2 * ROWS * EP;                            // [2][KC][UP] chunks of U rows
-  double* Cs = Ut + 2 * KC * UP;                              // [ROWS][UP] accumulated update
+  double* Cs = Ut;                                            // [ROWS][UP] accumulated update (after the loop)
   const int tid = threadIdx.x, lane = tid & 31;
   const int tsub = tid % TPR;
   const int rloc = tid / TPR;
@@ -197,7 +199,7 @@ __global__ void __launch_bounds__(256) sweep_panel_kernel(PanelArgs a) {
   const unsigned FULL = 0xffffffffu;
   const int base_lane = lane & ~(TPR - 1);
 
-  for (int e = tid; e < PW * PW; e += 256) {
+  for (int e = tid; e < PW * PW; e += PTHREADS) {
     const int r = e / PW, c = e % PW;
     Us[e] = (r < pw && c < pw && c >= r) ? a.U[(j0 + r) * n_in + j0 + c] : 0.0;
   }
@@ -209,8 +211,8 @@ __global__ void __launch_bounds__(256) sweep_panel_kernel(PanelArgs a) {
       const int64_t j = j0 + c;
       int64_t g = 0;
       if (a.gsz > 0) g = (a.static_groups && a.perm) ? clamp_idx(a.perm[j], n_in) / a.gsz : j / a.gsz;
-      ps[rloc * PW + c] = active ? a.scales[g * n_out + row] : 1.f;
-      pz[rloc * PW + c] = active ? a.zeros[g * n_out + row] : 0;
+      ps[c * ROWS + rloc] = active ? a.scales[g * n_out + row] : 1.f;
+      pz[c * ROWS + rloc] = active ? a.zeros[g * n_out + row] : 0;
     }
   }
   // The panel's running weights live in registers in fp64: each column of the panel
@@ -230,43 +232,46 @@ __global__ void __launch_bounds__(256) sweep_panel_kernel(PanelArgs a) {
   // GEMM per panel.  fp64 on the fp64 matrix units: warp w computes columns 8w..8w+7 of
   // the 16 x 64 product as two m8n8 tiles.
   if (a.j0 > a.o0) {
+    // Warp w computes rows 8w..8w+7 of the ROWS x 64 product as eight m8n8 tiles.
     const int g = lane >> 2, t = lane & 3, w = tid >> 5;
-    double acc[2][2] = {{0.0, 0.0}, {0.0, 0.0}};
+    double acc[PW / 8][2];
+#pragma unroll
+    for (int nb = 0; nb < PW / 8; ++nb) acc[nb][0] = acc[nb][1] = 0.0;
     const int nch = static_cast<int>((j0 - a.o0 + KC - 1) / KC);
-    // Chunk ch covers error columns [o0 + ch*KC, ...); both tiles are fetched with
-    // 16-byte cp.async (zero-filled outside the matrix), two chunks in flight.
     // 16-byte copies need even element offsets; odd panel widths (odd group sizes) take
     // the plain-load path.
     const bool vec_ok = ((j0 | a.o0 | n_in | static_cast<int64_t>(pw)) & 1) == 0;
+    // Chunk ch covers error columns [o0 + ch*KC, ...); both tiles are fetched with
+    // 16-byte cp.async (zero-filled outside the matrix), two chunks in flight.
     auto stage = [&](int ch, int buf) {
       const int64_t k0 = a.o0 + static_cast<int64_t>(ch) * KC;
+      double* es = Es + buf * ROWS * EP;
+      double* ut = Ut + buf * KC * UP;
       if (!vec_ok) {
-        for (int e = tid; e < ROWS * KC; e += 256) {
+        for (int e = tid; e < ROWS * KC; e += PTHREADS) {
           const int r = e / KC, k = e % KC;
           const int64_t gr = row0 + r, gk = k0 + k;
-          Es[buf * ROWS * EP + r * EP + k] = (gr < n_out && gk < j0) ? a.Err[gr * n_in + gk] : 0.0;
+          es[r * EP + k] = (gr < n_out && gk < j0) ? a.Err[gr * n_in + gk] : 0.0;
         }
-        for (int e = tid; e < KC * PW; e += 256) {
+        for (int e = tid; e < KC * PW; e += PTHREADS) {
           const int k = e / PW, c = e % PW;
           const int64_t gk = k0 + k;
-          Ut[buf * KC * UP + k * UP + c] = (gk < j0 && c < pw) ? a.U[gk * n_in + j0 + c] : 0.0;
+          ut[k * UP + c] = (gk < j0 && c < pw) ? a.U[gk * n_in + j0 + c] : 0.0;
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
         return;
       }
-      {
-        const int r = tid >> 4, kc = (tid & 15) * 2;  // 16 rows x 16 chunks
+      for (int e = tid; e < ROWS * (KC / 2); e += PTHREADS) {  // rows x 16-byte chunks
+        const int r = e / (KC / 2), kc = (e % (KC / 2)) * 2;
         const int64_t gr = row0 + r, gk = k0 + kc;
         const bool ok = gr < n_out && gk < j0;
-        cp_async16(Es + buf * ROWS * EP + r * EP + kc, ok ? a.Err + gr * n_in + gk : a.Err, ok);
+        cp_async16(es + r * EP + kc, ok ? a.Err + gr * n_in + gk : a.Err, ok);
       }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {                   // 32 rows x 32 chunks
-        const int e = tid + 256 * i;
-        const int k = e >> 5, c = (e & 31) * 2;
+      for (int e = tid; e < KC * (PW / 2); e += PTHREADS) {
+        const int k = e / (PW / 2), c = (e % (PW / 2)) * 2;
         const int64_t gk = k0 + k;
         const bool ok = gk < j0 && c < pw;
-        cp_async16(Ut + buf * KC * UP + k * UP + c, ok ? a.U + gk * n_in + j0 + c : a.U, ok);
+        cp_async16(ut + k * UP + c, ok ? a.U + gk * n_in + j0 + c : a.U, ok);
       }
       asm volatile("cp.async.commit_group;" ::: "memory");
     };
@@ -283,21 +288,21 @@ __global__ void __launch_bounds__(256) sweep_panel_kernel(PanelArgs a) {
       const double* ut = Ut + (ch & 1) * KC * UP;
 #pragma unroll
       for (int kk = 0; kk < KC; kk += 4) {
-        const double b0 = ut[(kk + t) * UP + w * 8 + g];
+        const double a0 = es[(w * 8 + g) * EP + kk + t];
 #pragma unroll
-        for (int mb = 0; mb < 2; ++mb) {
-          const double a0 = es[(mb * 8 + g) * EP + kk + t];
+        for (int nb = 0; nb < PW / 8; ++nb) {
+          const double b0 = ut[(kk + t) * UP + nb * 8 + g];
           asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
-                       : "+d"(acc[mb][0]), "+d"(acc[mb][1])
+                       : "+d"(acc[nb][0]), "+d"(acc[nb][1])
                        : "d"(a0), "d"(b0));
         }
       }
       __syncthreads();
     }
 #pragma unroll
-    for (int mb = 0; mb < 2; ++mb) {
-      Cs[(mb * 8 + g) * UP + w * 8 + 2 * t] = acc[mb][0];
-      Cs[(mb * 8 + g) * UP + w * 8 + 2 * t + 1] = acc[mb][1];
+    for (int nb = 0; nb < PW / 8; ++nb) {
+      Cs[(w * 8 + g) * UP + nb * 8 + 2 * t] = acc[nb][0];
+      Cs[(w * 8 + g) * UP + nb * 8 + 2 * t + 1] = acc[nb][1];
     }
     __syncthreads();
 #pragma unroll
@@ -344,8 +349,8 @@ __global__ void __launch_bounds__(256) sweep_panel_kernel(PanelArgs a) {
       double err = 0.0;
       if (tsub == o) {
         if (!a.in_panel_params) {
-          s = ps[rloc * PW + c];
-          z = pz[rloc * PW + c];
+          s = ps[c * ROWS + rloc];
+          z = pz[c * ROWS + rloc];
         }
         const double w = v[m];
         const int q = quant_code(static_cast<float>(w), s, z, maxq);
@@ -372,18 +377,18 @@ __global__ void __launch_bounds__(256) sweep_panel_kernel(PanelArgs a) {
   }
   __syncthreads();
   // codes: one ROWS-byte row segment per column
-  for (int e = tid; e < pw * ROWS; e += 256) {
+  for (int e = tid; e < pw * ROWS; e += PTHREADS) {
     const int c = e / ROWS, r = e % ROWS;
     if (row0 + r < n_out) a.codesT[(j0 + c) * n_out + row0 + r] = cs[c * ROWS + r];
   }
   if (!active) lsum = 0.0;
   for (int off = 16; off; off >>= 1) lsum += __shfl_xor_sync(FULL, lsum, off);
-  __shared__ double red[8];
+  __shared__ double red[PTHREADS / 32];
   if (lane == 0) red[tid >> 5] = lsum;
   __syncthreads();
   if (tid == 0) {
     double t = 0.0;
-    for (int i = 0; i < 8; ++i) t += red[i];
+    for (int i = 0; i < PTHREADS / 32; ++i) t += red[i];
     atomicAdd(a.loss, t);
   }
 }
@@ -535,7 +540,7 @@ int run_sweep(SweepArgs& a, cudaStream_t s, int* panel_width, int* outer_width) 
       pa.o0 = O0;
       pa.pw = static_cast<int>(p1 - p0);
       pa.in_panel_params = (dynamic_groups && g <= P) ? 1 : 0;
-      sweep_panel_kernel<<<panel_grid, 256, PANEL_SMEM, s>>>(pa);
+      sweep_panel_kernel<<<panel_grid, PTHREADS, PANEL_SMEM, s>>>(pa);
       GPTQ_TRY(after_launch());
     }
     if (O1 < n_in)  // every later column: W[:, O1:] -= Err[:, O0:O1] U[O0:O1, O1:]
