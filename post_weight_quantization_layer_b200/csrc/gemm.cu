@@ -284,7 +284,7 @@ int dgemm(cudaStream_t s, int64_t M, int64_t N, int64_t K, double alpha, const d
                       K % 2 == 0 && N % 2 == 0;
   if (mma_ok) {
     static cudaError_t attr = [] {
-      cudaError_t e[4] = {
+      cudaError_t e[6] = {
           cudaFuncSetAttribute(dgemm_mma_kernel<true, 128, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                DTile<128, 128>::SMEM),
           cudaFuncSetAttribute(dgemm_mma_kernel<false, 128, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -292,17 +292,32 @@ int dgemm(cudaStream_t s, int64_t M, int64_t N, int64_t K, double alpha, const d
           cudaFuncSetAttribute(dgemm_mma_kernel<true, 64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                DTile<64, 64>::SMEM),
           cudaFuncSetAttribute(dgemm_mma_kernel<false, 64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               DTile<64, 64>::SMEM)};
+                               DTile<64, 64>::SMEM),
+          cudaFuncSetAttribute(dgemm_mma_kernel<true, 32, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               DTile<32, 32>::SMEM),
+          cudaFuncSetAttribute(dgemm_mma_kernel<false, 32, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               DTile<32, 32>::SMEM)};
       for (cudaError_t x : e)
         if (x != cudaSuccess) return x;
       return cudaSuccess;
     }();
     if (attr != cudaSuccess) return GPTQ_ERR_CUDA;
-    // Small products: 64x64 tiles spread the work over 4x more SMs.
+    // Small products: 64x64 (or 32x32) tiles spread the work over 4x (16x) more SMs.
     const int64_t big_tiles = ((M + 127) / 128) * ((N + 127) / 128);
+    const int64_t mid_tiles = ((M + 63) / 64) * ((N + 63) / 64);
     const bool small = big_tiles < 2 * num_sms();
+    const bool tiny = mid_tiles < num_sms();
     const int u = upper ? 1 : 0;
-    if (small) {
+    if (tiny) {
+      dim3 g32(static_cast<unsigned>((N + 31) / 32), static_cast<unsigned>((M + 31) / 32));
+      if (g32.y > 65535u) return GPTQ_ERR_UNSUPPORTED;
+      if (transB)
+        dgemm_mma_kernel<true, 32, 32><<<g32, 256, DTile<32, 32>::SMEM, s>>>(M, N, K, alpha, A, lda, B, ldb, beta,
+                                                                            C, ldc, u, tri);
+      else
+        dgemm_mma_kernel<false, 32, 32><<<g32, 256, DTile<32, 32>::SMEM, s>>>(M, N, K, alpha, A, lda, B, ldb, beta,
+                                                                             C, ldc, u, tri);
+    } else if (small) {
       dim3 g64(static_cast<unsigned>((N + 63) / 64), static_cast<unsigned>((M + 63) / 64));
       if (g64.y > 65535u) return GPTQ_ERR_UNSUPPORTED;
       if (transB)

@@ -346,21 +346,21 @@ __global__ void __launch_bounds__(PTHREADS) sweep_panel_kernel(PanelArgs a) {
           a.zeros[(j / a.gsz) * n_out + row] = z;
         }
       }
-      double err = 0.0;
+      // All threads of the row take the decision on the owner's current value, so the
+      // chain carries one shuffle and no divergent branch; the owner keeps the error.
+      const double w = __shfl_sync(FULL, v[m], base_lane + o);
+      if (!a.in_panel_params) {
+        s = ps[c * ROWS + rloc];
+        z = pz[c * ROWS + rloc];
+      }
+      const int q = quant_code(static_cast<float>(w), s, z, maxq);
+      const double what = static_cast<double>(s) * static_cast<double>(q - z);
+      const double err = (w - what) * rdiag[c];
       if (tsub == o) {
-        if (!a.in_panel_params) {
-          s = ps[c * ROWS + rloc];
-          z = pz[c * ROWS + rloc];
-        }
-        const double w = v[m];
-        const int q = quant_code(static_cast<float>(w), s, z, maxq);
-        const double what = static_cast<double>(s) * static_cast<double>(q - z);
-        err = (w - what) * rdiag[c];
         v[m] = err;
         cs[c * ROWS + rloc] = static_cast<uint8_t>(q);
         lsum += err * err;
       }
-      err = __shfl_sync(FULL, err, base_lane + o);
 #pragma unroll
       for (int mm = m; mm < NCOL; ++mm) {
         const int col = tsub + TPR * mm;
