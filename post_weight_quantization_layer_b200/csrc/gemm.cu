@@ -154,8 +154,10 @@ __device__ __forceinline__ void dmma(double (&d)[2], double a, double b) {
                : "d"(a), "d"(b));
 }
 
+// At most 192 registers a thread (256 threads a CTA): one 128x128 CTA then leaves room on
+// its SM for one CTA of the sweep's panel kernel, which runs beside the trailing update.
 template <bool TRANSB, int BM, int BN>
-__global__ void __launch_bounds__(256, 1) dgemm_mma_kernel(int64_t M, int64_t N, int64_t K, double alpha,
+__global__ void __maxnreg__(192) dgemm_mma_kernel(int64_t M, int64_t N, int64_t K, double alpha,
                                                            const double* A, int64_t lda, const double* B,
                                                            int64_t ldb, double beta, double* C, int64_t ldc,
                                                            int upper, int tri) {
@@ -243,19 +245,29 @@ __global__ void __launch_bounds__(256, 1) dgemm_mma_kernel(int64_t M, int64_t N,
   }
   cp_async_wait<0>();
 
+  // Epilogue.  Each thread holds element pairs (gn, gn + 1) with gn even; N is even, so a
+  // pair is either wholly inside C or wholly outside, and 16-byte aligned.
+  // beta == 1 (the accumulating updates): fire-and-forget fp64 reductions, so the CTA does
+  // not wait on the latency of reading C; only this CTA writes these elements during the
+  // launch, so each one receives exactly one correctly rounded addition C + v.
 #pragma unroll
   for (int i = 0; i < MI; ++i) {
     const int64_t gm = m0 + wm * WM + i * 8 + g;
     if (gm >= M) continue;
 #pragma unroll
     for (int j = 0; j < NJ; ++j) {
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int64_t gn = n0 + wn * WN + j * 8 + 2 * t + e;
-        if (gn >= N) continue;
-        double* cp = C + gm * ldc + gn;
-        const double v = alpha * acc[i][j][e];
-        *cp = (beta == 0.0) ? v : fma(beta, *cp, v);
+      const int64_t gn = n0 + wn * WN + j * 8 + 2 * t;
+      if (gn >= N) continue;
+      double* cp = C + gm * ldc + gn;
+      const double v0 = alpha * acc[i][j][0], v1 = alpha * acc[i][j][1];
+      if (beta == 1.0) {
+        atomicAdd(cp, v0);
+        atomicAdd(cp + 1, v1);
+      } else if (beta == 0.0) {
+        *reinterpret_cast<double2*>(cp) = make_double2(v0, v1);
+      } else {
+        const double2 c = *reinterpret_cast<const double2*>(cp);
+        *reinterpret_cast<double2*>(cp) = make_double2(fma(beta, c.x, v0), fma(beta, c.y, v1));
       }
     }
   }
@@ -280,7 +292,7 @@ int dgemm(cudaStream_t s, int64_t M, int64_t N, int64_t K, double alpha, const d
   if (M <= 0 || N <= 0) return GPTQ_OK;
   dim3 grid(static_cast<unsigned>((N + TN - 1) / TN), static_cast<unsigned>((M + TM - 1) / TM));
   if (grid.y > 65535u) return GPTQ_ERR_UNSUPPORTED;
-  const bool mma_ok = aligned16(A) && aligned16(B) && aligned16(C) && lda % 2 == 0 && ldb % 2 == 0 &&
+  const bool mma_ok = aligned16(A) && aligned16(B) && aligned16(C) && lda % 2 == 0 && ldb % 2 == 0 && ldc % 2 == 0 &&
                       K % 2 == 0 && N % 2 == 0;
   if (mma_ok) {
     static cudaError_t attr = [] {
