@@ -141,6 +141,26 @@ int gptq_factor_hessian(const float* H, int64_t n_in, float damp_percent, int de
                         double* U, int32_t* perm, void* stream);
 
 /*
+ * gptq_factor_hessian for `count` independent Hessians at once (the distinct inputs of a
+ * decoder layer: attention input, attention output, MLP input, MLP down input), with the
+ * same arguments per item.  Source: as gptq_factor_hessian (chapter 5 §5.1.8).
+ *
+ * H[i], U[i], perm[i]: host arrays of `count` device pointers, each item laid out as in
+ * gptq_factor_hessian with its own order n_in[i] (host array).  Every item is factored
+ * exactly as gptq_factor_hessian would factor it (same kernels, bit-identical U and
+ * perm); the items run concurrently on library-owned streams forked from `stream` and
+ * joined back into it, the largest at the highest stream priority, so that the smaller
+ * factorisations fill the SMs that the largest one's serial steps leave idle.
+ * statuses: optional host array of `count` ints receiving each item's status.
+ * Returns GPTQ_OK when every item succeeded, else the first failing item's status
+ * (NOT_PD for a failed pivot; outputs of the other items are still valid).
+ * count <= 0 or a NULL array -> INVALID_ARG.  Blocking.
+ */
+int gptq_factor_hessians(int count, const float* const* H, const int64_t* n_in, float damp_percent,
+                         int desc_act, double* const* U, int32_t* const* perm, void* stream,
+                         int* statuses);
+
+/*
  * The sweep half: quantize W given the factor U and permutation perm produced
  * by gptq_factor_hessian (or any upper-triangular U with positive diagonal).
  * Arguments and outputs as in gptq_quantize_layer; U and perm are read-only.

@@ -13,6 +13,7 @@ from .api import (  # noqa: F401
     accumulate_hessian,
     device_status,
     factor_hessian,
+    factor_hessians,
     group_count,
     launch_count,
     quantize_layer,

@@ -42,6 +42,9 @@ _SIGNATURES = {
                                     c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                     ctypes.POINTER(GptqStats)]),
     "gptq_factor_hessian": (c_int, [c_void_p, c_i64, c_float, c_int, c_void_p, c_void_p, c_void_p]),
+    "gptq_factor_hessians": (c_int, [c_int, ctypes.POINTER(c_void_p), ctypes.POINTER(c_i64), c_float, c_int,
+                                     ctypes.POINTER(c_void_p), ctypes.POINTER(c_void_p), c_void_p,
+                                     ctypes.POINTER(c_int)]),
     "gptq_quantize_layer_factored": (c_int, [c_void_p, c_int, c_i64, c_i64, c_void_p, c_void_p, c_int, c_int,
                                              c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
                                              c_void_p, ctypes.POINTER(GptqStats)]),

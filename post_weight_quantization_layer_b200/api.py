@@ -121,6 +121,27 @@ def factor_hessian(H, damp_percent=0.01, desc_act=False, stream=None):
     return U, perm
 
 
+def factor_hessians(Hs, damp_percent=0.01, desc_act=False, stream=None):
+    """factor_hessian for several independent Hessians in one call (run concurrently by
+    the library).  Returns [(U, perm), ...] in the order of Hs; raises GPTQError naming
+    the first item that failed."""
+    Hs = list(Hs)
+    _need_cuda(*Hs)
+    k = len(Hs)
+    outs = [(torch.empty(H.shape[0], H.shape[0], dtype=torch.float64, device=H.device),
+             torch.empty(H.shape[0], dtype=torch.int32, device=H.device)) for H in Hs]
+    arr = ctypes.c_void_p * k
+    st_arr = (ctypes.c_int * k)()
+    st = lib().gptq_factor_hessians(k, arr(*[H.data_ptr() for H in Hs]),
+                                    (ctypes.c_int64 * k)(*[H.shape[0] for H in Hs]), float(damp_percent),
+                                    int(bool(desc_act)), arr(*[U.data_ptr() for U, _ in outs]),
+                                    arr(*[p.data_ptr() for _, p in outs]), _stream(stream), st_arr)
+    if st != OK:
+        bad = next((i for i in range(k) if st_arr[i] != OK), None)
+        _check(st, "gptq_factor_hessians" + (f" (item {bad})" if bad is not None else ""))
+    return outs
+
+
 def quantize_layer_factored(W, U, perm, bits=4, group_size=128, sym=True, static_groups=False, blocksize=128,
                             stats=False, out=None, stream=None) -> QuantResult:
     _need_cuda(W, U, perm)

@@ -3,6 +3,7 @@
 #include <cstring>
 #include <map>
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 
@@ -254,6 +255,61 @@ int gptq_factor_hessian(const float* H, int64_t n_in, float damp_percent, int de
     GPTQ_TRY(after_launch());
   }
   return finish(status, s);
+}
+
+int gptq_factor_hessians(int count, const float* const* H, const int64_t* n_in, float damp_percent,
+                         int desc_act, double* const* U, int32_t* const* perm, void* stream, int* statuses) {
+  if (count <= 0 || !H || !n_in || !U || !perm) return GPTQ_ERR_INVALID_ARG;
+  if (!valid_damp(damp_percent)) return GPTQ_ERR_INVALID_ARG;
+  for (int i = 0; i < count; ++i) {
+    if (!H[i] || !U[i] || !perm[i] || n_in[i] <= 0) return GPTQ_ERR_INVALID_ARG;
+    if (n_in[i] % 8 != 0 || n_in[i] > 65535) return GPTQ_ERR_UNSUPPORTED;
+    if (!aligned16(H[i]) || !aligned16(U[i]) || !aligned16(perm[i])) return GPTQ_ERR_UNSUPPORTED;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  size_t bytes = padded(static_cast<size_t>(count) * sizeof(int));
+  for (int i = 0; i < count; ++i) {
+    const size_t n = static_cast<size_t>(n_in[i]);
+    bytes += padded(factor_work_bytes(n_in[i])) + padded(factor_small_bytes(n_in[i])) + padded(n * 4);
+  }
+  Workspace ws;
+  GPTQ_TRY(alloc(ws, bytes + 256, s));
+  int* status = ws.take<int>(static_cast<size_t>(count));
+  GPTQ_CUDA(cudaMemsetAsync(status, 0, static_cast<size_t>(count) * sizeof(int), s));
+  // The largest factorisation is the critical path: its lane has the highest priority.
+  int largest = 0;
+  for (int i = 1; i < count; ++i)
+    if (n_in[i] > n_in[largest]) largest = i;
+  std::vector<LanePrio> prio(static_cast<size_t>(count), kLaneLow);
+  prio[static_cast<size_t>(largest)] = kLaneHigh;
+  {
+    LaneLease lanes(s);
+    GPTQ_TRY(lanes.acquire(count, prio.data()));
+    for (int i = 0; i < count; ++i) {
+      const int64_t n = n_in[i];
+      void* work = ws.take<char>(factor_work_bytes(n));
+      void* small = ws.take<char>(factor_small_bytes(n));
+      int32_t* invperm = ws.take<int32_t>(static_cast<size_t>(n));
+      cudaStream_t li = lanes[i].st;
+      GPTQ_TRY(factor_hessian(H[i], n, damp_percent, desc_act != 0, U[i], perm[i], invperm, work, small, status + i,
+                              li));
+      if (!desc_act) {
+        iota_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, li>>>(perm[i], n);
+        GPTQ_TRY(after_launch());
+      }
+    }
+  }  // every lane joins back into s
+  std::vector<int> h(static_cast<size_t>(count), 0);
+  if (cudaMemcpyAsync(h.data(), status, static_cast<size_t>(count) * sizeof(int), cudaMemcpyDeviceToHost, s) !=
+      cudaSuccess)
+    return GPTQ_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return GPTQ_ERR_CUDA;
+  int first = GPTQ_OK;
+  for (int i = 0; i < count; ++i) {
+    if (statuses) statuses[i] = h[static_cast<size_t>(i)];
+    if (first == GPTQ_OK && h[static_cast<size_t>(i)] != GPTQ_OK) first = h[static_cast<size_t>(i)];
+  }
+  return first;
 }
 
 int gptq_quantize_layer_factored(const void* W, int w_dtype, int64_t n_out, int64_t n_in, const double* U,

@@ -7,6 +7,8 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <utility>
+#include <vector>
 
 #include "../../include/gptq.h"
 
@@ -112,5 +114,29 @@ struct SweepArgs {
   cudaEvent_t ev[4];      // valid when stats != null
 };
 int run_sweep(SweepArgs& a, cudaStream_t s, int* panel_width, int* outer_width);
+
+// lanes.cu: library-owned streams leased by one call (see the file's header).
+enum LanePrio { kLaneHigh = 0, kLaneLow = 1 };
+struct Lane {
+  cudaStream_t st = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  cudaEvent_t aux = nullptr;  // free for the leasing call's own ordering
+};
+class LaneLease {
+ public:
+  explicit LaneLease(cudaStream_t s) : s_(s) {}
+  ~LaneLease();  // joins every lane into the caller's stream, returns the lanes
+  LaneLease(const LaneLease&) = delete;
+  LaneLease& operator=(const LaneLease&) = delete;
+  // Leases `count` lanes (priority class prio[i] for lane i), each forked from the
+  // caller's stream.
+  int acquire(int count, const LanePrio* prio);
+  Lane& operator[](int i) { return *lanes_[i].first; }
+
+ private:
+  cudaStream_t s_;
+  int dev_ = 0;
+  std::vector<std::pair<Lane*, int>> lanes_;
+};
 
 }  // namespace gptq

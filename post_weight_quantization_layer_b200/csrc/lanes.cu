@@ -1,0 +1,74 @@
+// Library-owned streams ("lanes") leased by one call for work that runs concurrently with
+// itself: the sweep's look-ahead (panels beside the trailing update) and the batched
+// factor (several Hessians at once).
+//
+// Lanes are created once per device and priority class and kept on a free list, so a call
+// pays no stream creation; concurrent calls from several host threads lease disjoint
+// lanes.  A lease forks every lane from the caller's stream (the lane starts after all
+// work already queued there) and, when it ends, makes the caller's stream wait for all
+// work issued on its lanes, on error paths too, so stream-ordered frees of the call's
+// workspace on the caller's stream never overtake a lane.
+#include <map>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+
+namespace gptq {
+namespace {
+
+std::mutex g_lane_mu;
+std::map<std::pair<int, int>, std::vector<Lane*>> g_lane_free;  // (device, priority class)
+
+int create_lane(LanePrio prio, Lane** out) {
+  int least = 0, greatest = 0;
+  if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) return GPTQ_ERR_CUDA;
+  Lane* l = new Lane;
+  bool ok = cudaStreamCreateWithPriority(&l->st, cudaStreamNonBlocking, prio == kLaneHigh ? greatest : least) ==
+            cudaSuccess;
+  for (cudaEvent_t* e : {&l->fork, &l->join, &l->aux})
+    ok = ok && cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess;
+  if (!ok) {
+    cudaGetLastError();
+    for (cudaEvent_t e : {l->fork, l->join, l->aux})
+      if (e) cudaEventDestroy(e);
+    if (l->st) cudaStreamDestroy(l->st);
+    delete l;
+    return GPTQ_ERR_CUDA;
+  }
+  *out = l;
+  return GPTQ_OK;
+}
+
+}  // namespace
+
+LaneLease::~LaneLease() {
+  for (auto& [l, prio] : lanes_) {
+    cudaEventRecord(l->join, l->st);
+    cudaStreamWaitEvent(s_, l->join, 0);
+  }
+  std::lock_guard<std::mutex> lk(g_lane_mu);
+  for (auto& [l, prio] : lanes_) g_lane_free[{dev_, prio}].push_back(l);
+}
+
+int LaneLease::acquire(int count, const LanePrio* prio) {
+  if (cudaGetDevice(&dev_) != cudaSuccess) return GPTQ_ERR_CUDA;
+  for (int i = 0; i < count; ++i) {
+    Lane* l = nullptr;
+    {
+      std::lock_guard<std::mutex> lk(g_lane_mu);
+      auto& v = g_lane_free[{dev_, static_cast<int>(prio[i])}];
+      if (!v.empty()) {
+        l = v.back();
+        v.pop_back();
+      }
+    }
+    if (!l) GPTQ_TRY(create_lane(prio[i], &l));
+    lanes_.emplace_back(l, static_cast<int>(prio[i]));
+    GPTQ_CUDA(cudaEventRecord(l->fork, s_));
+    GPTQ_CUDA(cudaStreamWaitEvent(l->st, l->fork, 0));
+  }
+  return GPTQ_OK;
+}
+
+}  // namespace gptq

@@ -31,9 +31,6 @@
 //   (latency-bound, one CTA of 4 warps per SM) shares the SMs with the GEMM's tiles
 //   (one CTA per SM), so the panels' time hides under the matrix-unit work.
 #include <algorithm>
-#include <map>
-#include <mutex>
-#include <vector>
 
 #include "common.cuh"
 
@@ -474,79 +471,6 @@ int stage_and_fixed(const SweepArgs& a, cudaStream_t s) {
   return GPTQ_OK;
 }
 
-// Library-owned streams for the look-ahead: a panel stream (highest priority) and a
-// trailing-update stream (lowest), with the events that order them.  Each sweep checks a
-// set out of a per-device free list, so concurrent calls from several host threads never
-// share one.
-struct SideStreams {
-  cudaStream_t panel = nullptr, gemm = nullptr;
-  cudaEvent_t fork = nullptr, pan = nullptr, rest = nullptr, join_p = nullptr, join_g = nullptr;
-};
-
-std::mutex g_side_mu;
-std::map<int, std::vector<SideStreams*>> g_side_free;
-
-int create_side(SideStreams** out) {
-  int least = 0, greatest = 0;
-  if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) return GPTQ_ERR_CUDA;
-  SideStreams* ss = new SideStreams;
-  bool ok = cudaStreamCreateWithPriority(&ss->panel, cudaStreamNonBlocking, greatest) == cudaSuccess &&
-            cudaStreamCreateWithPriority(&ss->gemm, cudaStreamNonBlocking, least) == cudaSuccess;
-  for (cudaEvent_t* e : {&ss->fork, &ss->pan, &ss->rest, &ss->join_p, &ss->join_g})
-    ok = ok && cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess;
-  if (!ok) {
-    cudaGetLastError();
-    for (cudaEvent_t e : {ss->fork, ss->pan, ss->rest, ss->join_p, ss->join_g})
-      if (e) cudaEventDestroy(e);
-    if (ss->panel) cudaStreamDestroy(ss->panel);
-    if (ss->gemm) cudaStreamDestroy(ss->gemm);
-    delete ss;
-    return GPTQ_ERR_CUDA;
-  }
-  *out = ss;
-  return GPTQ_OK;
-}
-
-// Checks a stream set out for one sweep; on destruction makes the caller's stream wait for
-// all work issued on the set (also on error paths, so that the workspace is never freed
-// under a running kernel) and returns the set to the free list.
-class SideLease {
- public:
-  SideLease(cudaStream_t s) : s_(s) {}
-  ~SideLease() {
-    if (!ss_) return;
-    cudaEventRecord(ss_->join_p, ss_->panel);
-    cudaEventRecord(ss_->join_g, ss_->gemm);
-    cudaStreamWaitEvent(s_, ss_->join_p, 0);
-    cudaStreamWaitEvent(s_, ss_->join_g, 0);
-    std::lock_guard<std::mutex> lk(g_side_mu);
-    g_side_free[dev_].push_back(ss_);
-  }
-  int acquire() {
-    if (cudaGetDevice(&dev_) != cudaSuccess) return GPTQ_ERR_CUDA;
-    {
-      std::lock_guard<std::mutex> lk(g_side_mu);
-      auto& v = g_side_free[dev_];
-      if (!v.empty()) {
-        ss_ = v.back();
-        v.pop_back();
-      }
-    }
-    if (!ss_) GPTQ_TRY(create_side(&ss_));
-    // fork: both side streams start after everything already queued on the caller's stream
-    GPTQ_CUDA(cudaEventRecord(ss_->fork, s_));
-    GPTQ_CUDA(cudaStreamWaitEvent(ss_->panel, ss_->fork, 0));
-    GPTQ_CUDA(cudaStreamWaitEvent(ss_->gemm, ss_->fork, 0));
-    return GPTQ_OK;
-  }
-  SideStreams* get() const { return ss_; }
-
- private:
-  cudaStream_t s_;
-  int dev_ = 0;
-  SideStreams* ss_ = nullptr;
-};
-
 }  // namespace
 
 int run_sweep(SweepArgs& a, cudaStream_t s, int* panel_width, int* outer_width) {
@@ -609,10 +533,11 @@ int run_sweep(SweepArgs& a, cudaStream_t s, int* panel_width, int* outer_width) 
   const unsigned panel_grid = static_cast<unsigned>((n_out + ROWS - 1) / ROWS);
 
   {
-    SideLease lease(s);
-    GPTQ_TRY(lease.acquire());
-    SideStreams* ss = lease.get();
-    cudaStream_t sp = ss->panel, sg = ss->gemm;
+    LaneLease lanes(s);
+    const LanePrio prio[2] = {kLaneHigh, kLaneLow};  // panels + look-ahead; trailing update
+    GPTQ_TRY(lanes.acquire(2, prio));
+    cudaStream_t sp = lanes[0].st, sg = lanes[1].st;
+    cudaEvent_t pan = lanes[0].aux, rest = lanes[1].aux;
     bool rest_issued = false;
     for (int64_t O0 = 0; O0 < n_in; O0 += Q) {
       const int64_t O1 = std::min(O0 + Q, n_in);
@@ -633,18 +558,18 @@ int run_sweep(SweepArgs& a, cudaStream_t s, int* panel_width, int* outer_width) 
       }
       if (O1 >= n_in) break;
       // Err[:, O0:O1] is complete: every later column gets W -= Err[:, O0:O1] U[O0:O1, :].
-      GPTQ_CUDA(cudaEventRecord(ss->pan, sp));
+      GPTQ_CUDA(cudaEventRecord(pan, sp));
       // The next block's columns first (on the panel stream, so its panels follow at once);
       // they were last written by the previous block's trailing update.
-      if (rest_issued) GPTQ_CUDA(cudaStreamWaitEvent(sp, ss->rest, 0));
+      if (rest_issued) GPTQ_CUDA(cudaStreamWaitEvent(sp, rest, 0));
       GPTQ_TRY(dgemm(sp, n_out, O2 - O1, O1 - O0, -1.0, a.Err + O0, n_in, a.U + O0 * n_in + O1, n_in, false, 1.0,
                      a.Wk + O1, n_in, false));
       // Every column after the next block, concurrently with the next block's panels.
       if (O2 < n_in) {
-        GPTQ_CUDA(cudaStreamWaitEvent(sg, ss->pan, 0));
+        GPTQ_CUDA(cudaStreamWaitEvent(sg, pan, 0));
         GPTQ_TRY(dgemm(sg, n_out, n_in - O2, O1 - O0, -1.0, a.Err + O0, n_in, a.U + O0 * n_in + O2, n_in, false,
                        1.0, a.Wk + O2, n_in, false));
-        GPTQ_CUDA(cudaEventRecord(ss->rest, sg));
+        GPTQ_CUDA(cudaEventRecord(rest, sg));
         rest_issued = true;
       }
     }

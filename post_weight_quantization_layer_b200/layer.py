@@ -2,9 +2,9 @@
 
 The modules that read the same input share one calibration Hessian (q/k/v the
 attention input, gate/up the MLP input; the OLMo quick-start's fused att_proj,
-§六 6.1).  Each distinct Hessian is accumulated once, factored once
-(gptq_factor_hessian), and every module that reads it is swept against that
-factor (gptq_quantize_layer_factored).  All arithmetic runs in the native
+§六 6.1).  Each distinct Hessian is accumulated once, factored once (all of them
+in one gptq_factor_hessians call, which runs them concurrently), and every module
+that reads it is swept against that factor (gptq_quantize_layer_factored).  All arithmetic runs in the native
 library; this module only sequences the calls and records per-phase CUDA-event
 times on the stream.
 """
@@ -69,7 +69,10 @@ def quantize_decoder_layer(acts, weights, modules, qcfg, hessians=None, timing=F
             launch_marks.append((a, b))
             Hs[h] = H
         m_h = mark()
-        factors = {h: api.factor_hessian(H, qcfg.damp_percent, qcfg.desc_act, stream=stream) for h, H in Hs.items()}
+        # every distinct Hessian factored in one call: the library runs them concurrently
+        keys = list(Hs)
+        factors = dict(zip(keys, api.factor_hessians([Hs[h] for h in keys], qcfg.damp_percent, qcfg.desc_act,
+                                                     stream=stream)))
         m_f = mark()
         results = {}
         for mod in modules:

@@ -62,3 +62,32 @@ def test_act_order_ties_are_stable():
     H = torch.diag(d)
     _, perm = gq.factor_hessian(H.to(dev), 0.01, True)
     assert perm.cpu().tolist() == sorted(range(8), key=lambda i: (-float(d[i]), i))
+
+
+@pytest.mark.parametrize("desc_act", [False, True])
+def test_batched_factor_is_bit_identical_to_single_calls(desc_act):
+    """Concurrent factorisation of several Hessians gives exactly the single-call results."""
+    dev = device()
+    Hs = [_h(n, T, 7 * n + T).to(dev) for n, T in [(1032, 4096), (256, 512), (520, 1500), (264, 2000)]]
+    outs = gq.factor_hessians(Hs, 0.01, desc_act)
+    torch.cuda.synchronize()
+    for H, (U, perm) in zip(Hs, outs):
+        U1, p1 = gq.factor_hessian(H, 0.01, desc_act)
+        torch.cuda.synchronize()
+        assert torch.equal(perm, p1)
+        assert torch.equal(U, U1)
+
+
+def test_batched_factor_reports_the_failing_item():
+    dev = device()
+    good = _h(256, 512, 11).to(dev)
+    bad = -torch.eye(128, device=dev)
+    with pytest.raises(gq.GPTQError) as e:
+        gq.factor_hessians([good, bad], 0.01, True)
+    assert e.value.status == 3 and "item 1" in str(e.value)
+    # after a failing batch the context stays usable and batched results still match
+    outs = gq.factor_hessians([good, good * 2], 0.01, True)
+    torch.cuda.synchronize()
+    U1, _ = gq.factor_hessian(good, 0.01, True)
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0][0], U1)

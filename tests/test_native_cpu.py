@@ -93,6 +93,24 @@ def test_factor_rejections(L):
     assert q(FAKE, 1, 64, 256, FAKE, FAKE, 6, 128, 1, 0, 128, FAKE, FAKE, FAKE, FAKE, None, None) == INVALID
 
 
+def test_batched_factor_rejections(L):
+    f = L.gptq_factor_hessians
+    P = ctypes.c_void_p * 2
+    ptrs = P(FAKE, FAKE)
+    ns = (ctypes.c_int64 * 2)(64, 128)
+    st = (ctypes.c_int * 2)()
+    assert f(0, ptrs, ns, 0.01, 0, ptrs, ptrs, None, st) == INVALID
+    assert f(-1, ptrs, ns, 0.01, 0, ptrs, ptrs, None, st) == INVALID
+    assert f(2, None, ns, 0.01, 0, ptrs, ptrs, None, st) == INVALID
+    assert f(2, ptrs, None, 0.01, 0, ptrs, ptrs, None, st) == INVALID
+    assert f(2, ptrs, ns, 0.0, 0, ptrs, ptrs, None, st) == INVALID
+    assert f(2, ptrs, ns, math.nan, 0, ptrs, ptrs, None, st) == INVALID
+    assert f(2, P(FAKE, None), ns, 0.01, 0, ptrs, ptrs, None, st) == INVALID
+    assert f(2, ptrs, (ctypes.c_int64 * 2)(64, 0), 0.01, 0, ptrs, ptrs, None, st) == INVALID
+    assert f(2, ptrs, (ctypes.c_int64 * 2)(64, 60), 0.01, 0, ptrs, ptrs, None, st) == UNSUPPORTED
+    assert f(2, P(FAKE, MISALIGNED), ns, 0.01, 0, ptrs, ptrs, None, st) == UNSUPPORTED
+
+
 def test_python_binding_fails_loudly_without_cuda_tensors():
     import torch
 
