@@ -8,7 +8,11 @@
 // Design (sm_100a):
 // * Output tiles of 128 (rows i) x 256 (cols j) of H; only tiles touching the upper
 //   triangle are computed and each element is added to both H[i][j] and H[j][i].
-// * Split-K over tokens: grid = tiles x splits; every CTA owns one (tile, token range).
+// * Persistent grid, one CTA per SM, walking (tile, token segment) units in the order of
+//   hessian_sched.cuh: each wave of CTAs works on one token segment of a compact group of
+//   tiles, so the CTAs stream the same token rows in step and each row of X is fetched
+//   from DRAM a few times instead of once per tile; a CTA's consecutive units of one
+//   tile accumulate without write-back, and its epilogue overlaps its next unit's MMAs.
 // * A warp-specialised CTA of 10 warps: warp 0 issues TMA loads of X (channels
 //   contiguous, 128-byte swizzle) into a 4-stage shared-memory ring; warp 1 issues
 //   tcgen05.mma kind::f16 (A and B both MN-major, since X^T and X come from the
@@ -23,6 +27,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "hessian_sched.cuh"
 #include "sm100.cuh"
 
 namespace gptq {
@@ -45,26 +50,10 @@ constexpr uint32_t WAIT_LIMIT = 1u << 24;
 
 __device__ int g_hessian_status = 0;
 
-__device__ __forceinline__ void tile_coords(int t, int n, int& bi, int& bj) {
-  const int rb = (n + BM - 1) / BM;
-  const int cb = (n + BN - 1) / BN;
-  for (int j = 0; j < cb; ++j) {
-    const int cnt = min(rb, 2 * j + 2);  // row blocks with bi*128 <= j*256 + 255
-    if (t < cnt) {
-      bi = t;
-      bj = j;
-      return;
-    }
-    t -= cnt;
-  }
-  bi = 0;
-  bj = 0;
-}
-
 template <uint32_t AB_FMT>
 __global__ void __launch_bounds__(THREADS, 1)
     hessian_syrk_kernel(const __grid_constant__ CUtensorMap tmap, float* __restrict__ H, int n, int64_t T,
-                        int tiles, int64_t tok_per_split) {
+                        int tiles, int S, int64_t tok_per_seg) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
@@ -75,15 +64,16 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = blockIdx.x / tiles, tile = blockIdx.x % tiles;
-  int bi, bj;
-  tile_coords(tile, n, bi, bj);
-  const int i0 = bi * BM, j0 = bj * BN;
-  const int64_t t0 = static_cast<int64_t>(split) * tok_per_split;
-  const int64_t t1 = min(T, t0 + tok_per_split);
-  const int nk = t1 > t0 ? static_cast<int>((t1 - t0 + BK - 1) / BK) : 0;
-  if (nk == 0) return;  // uniform over the CTA, before any barrier or TMEM use
-  const int nchunks = (nk + FLUSH_KSTEPS - 1) / FLUSH_KSTEPS;
+  const int G = static_cast<int>(gridDim.x);
+  const int units = tiles * S;  // < 2^31 (checked on the host)
+  // k-steps of unit u (uniform over the CTA)
+  auto unit_ksteps = [&](int u, int& tile, int64_t& t0) {
+    int seg;
+    hsched::unit_at(u, tiles, S, G, tile, seg);
+    t0 = static_cast<int64_t>(seg) * tok_per_seg;
+    const int64_t t1 = min(T, t0 + tok_per_seg);
+    return t1 > t0 ? static_cast<int>((t1 - t0 + BK - 1) / BK) : 0;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -114,22 +104,30 @@ __global__ void __launch_bounds__(THREADS, 1)
       int stage = 0;
       uint32_t ph = 0;
       int issued = 0;
-      for (int ks = 0; ks < nk; ++ks) {
-        if (!mbar_wait(&empty[stage], ph ^ 1u, WAIT_LIMIT)) {
-          ok = false;
-          break;
-        }
-        uint8_t* sa = smem + stage * STAGE_BYTES;
-        mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-        const int y = static_cast<int>(t0 + static_cast<int64_t>(ks) * BK);
-        tma_load_2d(sa, &tmap, &full[stage], i0, y);
-        tma_load_2d(sa + BOX_BYTES, &tmap, &full[stage], i0 + 64, y);
+      for (int u = blockIdx.x; u < units && ok; u += G) {
+        int tile;
+        int64_t t0;
+        const int nk = unit_ksteps(u, tile, t0);
+        int bi, bj;
+        hsched::tile_at(tile, n, bi, bj);
+        const int i0 = bi * BM, j0 = bj * BN;
+        for (int ks = 0; ks < nk; ++ks) {
+          if (!mbar_wait(&empty[stage], ph ^ 1u, WAIT_LIMIT)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+          const int y = static_cast<int>(t0 + static_cast<int64_t>(ks) * BK);
+          tma_load_2d(sa, &tmap, &full[stage], i0, y);
+          tma_load_2d(sa + BOX_BYTES, &tmap, &full[stage], i0 + 64, y);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) tma_load_2d(sa + A_BYTES + q * BOX_BYTES, &tmap, &full[stage], j0 + 64 * q, y);
-        ++issued;
-        if (++stage == STAGES) {
-          stage = 0;
-          ph ^= 1u;
+          for (int q = 0; q < 4; ++q) tma_load_2d(sa + A_BYTES + q * BOX_BYTES, &tmap, &full[stage], j0 + 64 * q, y);
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            ph ^= 1u;
+          }
         }
       }
       // Before leaving, make sure no copy of ours is still landing in shared memory
@@ -150,38 +148,45 @@ __global__ void __launch_bounds__(THREADS, 1)
       constexpr uint32_t idesc = instr_desc(AB_FMT, true, true, BM, BN);
       int stage = 0;
       uint32_t ph = 0;
-      int ks = 0;
-      for (int c = 0; c < nchunks && ok; ++c) {
-        const int b = c & 1;
-        if (!mbar_wait(&acce[b], ((c >> 1) & 1) ^ 1u, WAIT_LIMIT)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t dcol = tmem + static_cast<uint32_t>(b * BN);
-        const int kend = min(nk, ks + FLUSH_KSTEPS);
-        for (int s_in = 0; ks < kend; ++ks, ++s_in) {
-          if (!mbar_wait(&full[stage], ph, WAIT_LIMIT)) {
+      int cg = 0;  // chunks issued by this CTA so far (selects the TMEM buffer and its phase)
+      for (int u = blockIdx.x; u < units && ok; u += G) {
+        int tile;
+        int64_t t0;
+        const int nk = unit_ksteps(u, tile, t0);
+        const int nchunks = (nk + FLUSH_KSTEPS - 1) / FLUSH_KSTEPS;
+        int ks = 0;
+        for (int c = 0; c < nchunks && ok; ++c, ++cg) {
+          const int b = cg & 1;
+          if (!mbar_wait(&acce[b], ((cg >> 1) & 1) ^ 1u, WAIT_LIMIT)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
-          const uint32_t sb = sa + A_BYTES;
+          const uint32_t dcol = tmem + static_cast<uint32_t>(b * BN);
+          const int kend = min(nk, ks + FLUSH_KSTEPS);
+          for (int s_in = 0; ks < kend; ++ks, ++s_in) {
+            if (!mbar_wait(&full[stage], ph, WAIT_LIMIT)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+            const uint32_t sb = sa + A_BYTES;
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            // 16 tokens = two 8-row swizzle atoms = 2048 bytes along K.
-            const uint64_t ad = smem_desc_sw128(sa + k * 2048, BOX_BYTES, 1024);
-            const uint64_t bd = smem_desc_sw128(sb + k * 2048, BOX_BYTES, 1024);
-            umma_f16(dcol, ad, bd, idesc, (s_in > 0 || k > 0) ? 1u : 0u);
+            for (int k = 0; k < BK / 16; ++k) {
+              // 16 tokens = two 8-row swizzle atoms = 2048 bytes along K.
+              const uint64_t ad = smem_desc_sw128(sa + k * 2048, BOX_BYTES, 1024);
+              const uint64_t bd = smem_desc_sw128(sb + k * 2048, BOX_BYTES, 1024);
+              umma_f16(dcol, ad, bd, idesc, (s_in > 0 || k > 0) ? 1u : 0u);
+            }
+            umma_commit(&empty[stage]);
+            if (++stage == STAGES) {
+              stage = 0;
+              ph ^= 1u;
+            }
           }
-          umma_commit(&empty[stage]);
-          if (++stage == STAGES) {
-            stage = 0;
-            ph ^= 1u;
-          }
+          umma_commit(&accf[b]);
         }
-        umma_commit(&accf[b]);
       }
       umma_commit(done);
       mbar_wait(done, 0, WAIT_LIMIT);
@@ -193,45 +198,66 @@ __global__ void __launch_bounds__(THREADS, 1)
     float acc[128];
 #pragma unroll
     for (int i = 0; i < 128; ++i) acc[i] = 0.f;
-    for (int c = 0; c < nchunks; ++c) {
-      const int b = c & 1;
-      if (!mbar_wait(&accf[b], (c >> 1) & 1, WAIT_LIMIT)) {
-        ok = false;
-        break;
+    int cg = 0;
+    for (int u = blockIdx.x; u < units && ok; u += G) {
+      int tile;
+      int64_t t0;
+      const int nk = unit_ksteps(u, tile, t0);
+      const int nchunks = (nk + FLUSH_KSTEPS - 1) / FLUSH_KSTEPS;
+      for (int c = 0; c < nchunks; ++c, ++cg) {
+        const int b = cg & 1;
+        if (!mbar_wait(&accf[b], (cg >> 1) & 1, WAIT_LIMIT)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float v[32];
+          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(b * BN + half * 128 + q * 32), v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) acc[q * 32 + i] += v[i];
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acce[b]);
       }
-      tc_fence_after();
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float v[32];
-        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(b * BN + half * 128 + q * 32), v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) acc[q * 32 + i] += v[i];
+      if (!ok) break;
+      // Write the tile back once this CTA's next unit belongs to another tile (or there is
+      // none); the MMA warp meanwhile fills the TMEM buffer just released.
+      bool flush = true;
+      if (u + G < units) {
+        int ntile, nseg;
+        hsched::unit_at(u + G, tiles, S, G, ntile, nseg);
+        flush = ntile != tile;
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acce[b]);
-    }
-    const int gi = i0 + quad * 32 + lane;
-    const int jb = j0 + half * 128;
-    if (ok && gi < n) {
-      float* rowp = H + static_cast<size_t>(gi) * n;
+      if (!flush) continue;
+      int bi, bj;
+      hsched::tile_at(tile, n, bi, bj);
+      const int gi = bi * BM + quad * 32 + lane;
+      const int jb = bj * BN + half * 128;
+      if (gi < n) {
+        float* rowp = H + static_cast<size_t>(gi) * n;
 #pragma unroll
-      for (int c4 = 0; c4 < 32; ++c4) {
-        const int gj = jb + c4 * 4;
-        if (gj >= gi && gj + 3 < n) {
-          atomicAdd(reinterpret_cast<float4*>(rowp + gj),
-                    make_float4(2.f * acc[4 * c4], 2.f * acc[4 * c4 + 1], 2.f * acc[4 * c4 + 2], 2.f * acc[4 * c4 + 3]));
-        } else {
+        for (int c4 = 0; c4 < 32; ++c4) {
+          const int gj = jb + c4 * 4;
+          if (gj >= gi && gj + 3 < n) {
+            atomicAdd(reinterpret_cast<float4*>(rowp + gj),
+                      make_float4(2.f * acc[4 * c4], 2.f * acc[4 * c4 + 1], 2.f * acc[4 * c4 + 2], 2.f * acc[4 * c4 + 3]));
+          } else {
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            if (gj + e < n && gj + e >= gi) atomicAdd(rowp + gj + e, 2.f * acc[4 * c4 + e]);
+            for (int e = 0; e < 4; ++e)
+              if (gj + e < n && gj + e >= gi) atomicAdd(rowp + gj + e, 2.f * acc[4 * c4 + e]);
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const int gj = jb + c;
+          if (gj < n && gj > gi) atomicAdd(H + static_cast<size_t>(gj) * n + gi, 2.f * acc[c]);
         }
       }
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        const int gj = jb + c;
-        if (gj < n && gj > gi) atomicAdd(H + static_cast<size_t>(gj) * n + gi, 2.f * acc[c]);
-      }
+      for (int i = 0; i < 128; ++i) acc[i] = 0.f;
     }
   }
   if (!ok) atomicExch(&g_hessian_status, kStatusTimeout);
@@ -261,29 +287,27 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-int count_tiles(int n) {
-  const int rb = (n + BM - 1) / BM, cb = (n + BN - 1) / BN;
-  int t = 0;
-  for (int j = 0; j < cb; ++j) t += std::min(rb, 2 * j + 2);
-  return t;
-}
-
-// Token splits: balance (tiles x splits) over the SMs while keeping every unit long
-// enough to amortise its prologue (about ten k-steps' worth of time).
-int choose_splits(int tiles, int64_t ksteps, int sms) {
+// Token segments per tile.  The persistent grid runs G = min(SMs, units) CTAs; full tile
+// groups take S rounds each and the last group's g*S units take ceil(g*S/G) rounds.  Pick
+// the S that keeps the SMs busiest while every unit stays long enough to amortise its
+// start (about ten k-steps' worth).
+int choose_segments(int tiles, int64_t ksteps, int sms) {
   int best = 1;
   double best_score = -1.0;
   const int smax = static_cast<int>(std::min<int64_t>(ksteps, 1024));
-  for (int s = 1; s <= smax; ++s) {
-    const int64_t kper = (ksteps + s - 1) / s;
-    if (s > 1 && kper < 16) break;
-    const int64_t units = static_cast<int64_t>(tiles) * s;
-    const int64_t waves = (units + sms - 1) / sms;
-    const double eff = static_cast<double>(units) / static_cast<double>(waves * sms);
+  for (int S = 1; S <= smax; ++S) {
+    const int64_t kper = (ksteps + S - 1) / S;
+    if (S > 1 && kper < 16) break;
+    const int64_t units = static_cast<int64_t>(tiles) * S;
+    const int64_t G = std::min<int64_t>(sms, units);
+    const int64_t full = tiles / G, g = tiles % G;
+    const int64_t rounds = full * S + (g * S + G - 1) / G;
+    const double eff = static_cast<double>(units) / static_cast<double>(rounds * G) *
+                       static_cast<double>(G) / static_cast<double>(sms);
     const double score = eff * static_cast<double>(kper) / static_cast<double>(kper + 10);
     if (score > best_score + 1e-9) {
       best_score = score;
-      best = s;
+      best = S;
     }
   }
   return best;
@@ -299,7 +323,7 @@ int launch_impl(const void* X, int64_t T, int n, float* H, cudaStream_t st) {
     attr_err = cudaFuncSetAttribute(hessian_syrk_kernel<F>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return GPTQ_ERR_CUDA;
-  const int tiles = count_tiles(n);
+  const int tiles = hsched::tile_count(n);
   const int sms = num_sms();
   // TMA coordinates are 32-bit: walk very long token streams in chunks.
   const int64_t CH = int64_t(1) << 30;
@@ -316,11 +340,12 @@ int launch_impl(const void* X, int64_t T, int n, float* H, cudaStream_t st) {
                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return GPTQ_ERR_CUDA;
     const int64_t ksteps = (Tc + BK - 1) / BK;
-    const int splits0 = choose_splits(tiles, ksteps, sms);
-    const int64_t kper = (ksteps + splits0 - 1) / splits0;
-    const int64_t tok_per_split = kper * BK;
-    const int splits = static_cast<int>((Tc + tok_per_split - 1) / tok_per_split);
-    hessian_syrk_kernel<F><<<tiles * splits, THREADS, SMEM_BYTES, st>>>(tm, H, n, Tc, tiles, tok_per_split);
+    const int S0 = choose_segments(tiles, ksteps, sms);
+    const int64_t tok_per_seg = ((ksteps + S0 - 1) / S0) * BK;
+    const int S = static_cast<int>((Tc + tok_per_seg - 1) / tok_per_seg);  // no empty segments
+    if (static_cast<int64_t>(tiles) * S >= (int64_t(1) << 31)) return GPTQ_ERR_UNSUPPORTED;
+    const int G = static_cast<int>(std::min<int64_t>(sms, static_cast<int64_t>(tiles) * S));
+    hessian_syrk_kernel<F><<<G, THREADS, SMEM_BYTES, st>>>(tm, H, n, Tc, tiles, S, tok_per_seg);
     GPTQ_TRY(after_launch());
   }
   return GPTQ_OK;

@@ -26,7 +26,7 @@ def _gpu_h(X, n, chunks=1):
 
 
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
-@pytest.mark.parametrize("T,n", [(777, 264), (64, 8), (130, 392), (1500, 520)])
+@pytest.mark.parametrize("T,n", [(777, 264), (64, 8), (130, 392), (1500, 520), (777, 4104), (5000, 1032)])
 def test_integer_valued_x_is_bit_exact(dtype, T, n):
     """Entries in {-3..3} are exact in fp16/bf16 and every partial sum stays below
     2^24, so the fp32 result must equal the integer SYRK exactly (both triangles)."""
