@@ -113,7 +113,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu_id), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
         except Exception:
@@ -255,9 +255,13 @@ def run_native(args, world, rank, local):
         "algorithmic_flops_per_launch": work["hessian_flops"],
         "per_launch_tflops": [round(x, 1) for x in per_launch],
     }
-    traffic = load_traffic()
-    if traffic is not None:
-        roofline["traffic"] = traffic
+    traffic = load_traffic() if args.config == "llama7b" and T == cfg.tokens else None
+    if traffic is not None and len(traffic) == len(launch_ms):
+        # per launch, like `achieved` (the mean over this layer's Hessian launches)
+        roofline["traffic"] = round(statistics.mean(traffic))
+        roofline["traffic_per_launch"] = traffic
+        roofline["traffic_source"] = "ncu dram__bytes_read.sum + dram__bytes_write.sum, " \
+                                     "profiles/hessian_syrk_dram_llama7b_layer.md"
 
     phases = {
         "hessian": {"ms": round(h_ms, 3), "tflops": round(h_tflops, 1),
@@ -324,13 +328,17 @@ def measure_fp64_peak(dev):
 
 
 def load_traffic():
-    """DRAM traffic per Hessian launch from the committed ncu summary, if present."""
-    path = os.path.join(ROOT, "profiles", "hessian_traffic.json")
+    """DRAM bytes (read + write) per Hessian launch of one decoder layer, from the committed
+    ncu summary of the same bench command (profiles/hessian_syrk_dram_llama7b_layer.md)."""
+    path = os.path.join(ROOT, "profiles", "hessian_syrk_dram_llama7b_layer.md")
     try:
         with open(path) as f:
-            return json.load(f)
-    except Exception:
-        return None
+            for ln in f:
+                if ln.startswith("traffic_bytes_per_launch:"):
+                    return [float(x) for x in ln.split(":", 1)[1].strip().strip("[]").split(",")]
+    except OSError:
+        pass
+    return None
 
 
 def run_e2e(args, cfg, acts, weights, dev, stream, world, Hbuf):
