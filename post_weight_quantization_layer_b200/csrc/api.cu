@@ -188,6 +188,26 @@ int sweep_common(const void* W, int w_dtype, int64_t n_out, int64_t n_in, const 
   return GPTQ_OK;
 }
 
+// The factor of one Hessian on leased lanes: the recursion on a lane of priority `prio`, the
+// top level's T product on a low-priority lane beside it (so it fills the SMs that the left
+// half's serial leaf steps leave idle).  Both lanes join back into s when this returns.
+// `work` must hold factor_work_bytes(n, true).
+int factor_on_lanes(const float* H, int64_t n, float damp, bool desc_act, double* U, int32_t* perm,
+                    int32_t* invperm, void* work, void* small, int* status, bool fill_identity, LanePrio prio,
+                    cudaStream_t s) {
+  LaneLease lanes(s);
+  const LanePrio pr[2] = {prio, kLaneLow};
+  GPTQ_TRY(lanes.acquire(2, pr));
+  cudaStream_t main = lanes[0].st;
+  GPTQ_TRY(factor_hessian(H, n, damp, desc_act, U, perm, invperm, work, small, status, main, lanes[1].st,
+                          lanes[1].aux, lanes[1].aux2));
+  if (fill_identity && !desc_act) {
+    iota_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, main>>>(perm, n);
+    GPTQ_TRY(after_launch());
+  }
+  return GPTQ_OK;
+}
+
 }  // namespace
 }  // namespace gptq
 
@@ -243,17 +263,14 @@ int gptq_factor_hessian(const float* H, int64_t n_in, float damp_percent, int de
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t n = static_cast<size_t>(n_in);
   Workspace ws;
-  GPTQ_TRY(alloc(ws, padded(factor_work_bytes(n_in)) + padded(factor_small_bytes(n_in)) + padded(n * 4) + 512, s));
-  void* work = ws.take<char>(factor_work_bytes(n_in));
+  GPTQ_TRY(alloc(ws, padded(factor_work_bytes(n_in, true)) + padded(factor_small_bytes(n_in)) + padded(n * 4) + 512, s));
+  void* work = ws.take<char>(factor_work_bytes(n_in, true));
   void* small = ws.take<char>(factor_small_bytes(n_in));
   int32_t* invperm = ws.take<int32_t>(n);
   int* status = ws.take<int>(1);
   GPTQ_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
-  GPTQ_TRY(factor_hessian(H, n_in, damp_percent, desc_act != 0, U, perm, invperm, work, small, status, s));
-  if (!desc_act) {
-    iota_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(perm, n_in);
-    GPTQ_TRY(after_launch());
-  }
+  GPTQ_TRY(factor_on_lanes(H, n_in, damp_percent, desc_act != 0, U, perm, invperm, work, small, status, true,
+                           kLaneHigh, s));
   return finish(status, s);
 }
 
@@ -270,31 +287,33 @@ int gptq_factor_hessians(int count, const float* const* H, const int64_t* n_in, 
   size_t bytes = padded(static_cast<size_t>(count) * sizeof(int));
   for (int i = 0; i < count; ++i) {
     const size_t n = static_cast<size_t>(n_in[i]);
-    bytes += padded(factor_work_bytes(n_in[i])) + padded(factor_small_bytes(n_in[i])) + padded(n * 4);
+    bytes += padded(factor_work_bytes(n_in[i], true)) + padded(factor_small_bytes(n_in[i])) + padded(n * 4);
   }
   Workspace ws;
   GPTQ_TRY(alloc(ws, bytes + 256, s));
   int* status = ws.take<int>(static_cast<size_t>(count));
   GPTQ_CUDA(cudaMemsetAsync(status, 0, static_cast<size_t>(count) * sizeof(int), s));
-  // The largest factorisation is the critical path: its lane has the highest priority.
+  // The largest factorisation is the critical path: its lanes have the highest priority.
   int largest = 0;
   for (int i = 1; i < count; ++i)
     if (n_in[i] > n_in[largest]) largest = i;
-  std::vector<LanePrio> prio(static_cast<size_t>(count), kLaneLow);
-  prio[static_cast<size_t>(largest)] = kLaneHigh;
+  // Two lanes per item: its recursion, and its top-level T product beside it.
+  std::vector<LanePrio> prio(2 * static_cast<size_t>(count), kLaneLow);
+  prio[2 * static_cast<size_t>(largest)] = kLaneHigh;
   {
     LaneLease lanes(s);
-    GPTQ_TRY(lanes.acquire(count, prio.data()));
+    GPTQ_TRY(lanes.acquire(2 * count, prio.data()));
     for (int i = 0; i < count; ++i) {
       const int64_t n = n_in[i];
-      void* work = ws.take<char>(factor_work_bytes(n));
+      void* work = ws.take<char>(factor_work_bytes(n, true));
       void* small = ws.take<char>(factor_small_bytes(n));
       int32_t* invperm = ws.take<int32_t>(static_cast<size_t>(n));
-      cudaStream_t li = lanes[i].st;
+      Lane& li = lanes[2 * i];
+      Lane& lt = lanes[2 * i + 1];
       GPTQ_TRY(factor_hessian(H[i], n, damp_percent, desc_act != 0, U[i], perm[i], invperm, work, small, status + i,
-                              li));
+                              li.st, lt.st, lt.aux, lt.aux2));
       if (!desc_act) {
-        iota_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, li>>>(perm[i], n);
+        iota_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, li.st>>>(perm[i], n);
         GPTQ_TRY(after_launch());
       }
     }
@@ -364,10 +383,10 @@ int gptq_quantize_layer(const void* W, int w_dtype, int64_t n_out, int64_t n_in,
   GPTQ_TRY(evs.create(stats != nullptr));
   Workspace ws;
   GPTQ_TRY(alloc(ws,
-                 padded(factor_work_bytes(n_in)) + padded(ni * ni * 8) + padded(factor_small_bytes(n_in)) +
+                 padded(factor_work_bytes(n_in, true)) + padded(ni * ni * 8) + padded(factor_small_bytes(n_in)) +
                      2 * padded(ni * 4) + 2 * padded(no * ni * 8) + padded(no * ni) + 1024,
                  s));
-  void* work = ws.take<char>(factor_work_bytes(n_in));
+  void* work = ws.take<char>(factor_work_bytes(n_in, true));
   double* U = ws.take<double>(ni * ni);
   void* small = ws.take<char>(factor_small_bytes(n_in));
   int32_t* perm = ws.take<int32_t>(ni);
@@ -379,7 +398,8 @@ int gptq_quantize_layer(const void* W, int w_dtype, int64_t n_out, int64_t n_in,
   int* status = ws.take<int>(1);
   GPTQ_CUDA(cudaMemsetAsync(status, 0, sizeof(int), s));
   if (evs.on) GPTQ_CUDA(cudaEventRecord(evs.ev[4], s));
-  GPTQ_TRY(factor_hessian(H, n_in, damp_percent, desc_act != 0, U, perm, invperm, work, small, status, s));
+  GPTQ_TRY(factor_on_lanes(H, n_in, damp_percent, desc_act != 0, U, perm, invperm, work, small, status, false,
+                           kLaneHigh, s));
   if (evs.on) GPTQ_CUDA(cudaEventRecord(evs.ev[5], s));
   GPTQ_TRY(sweep_common(W, w_dtype, n_out, n_in, U, desc_act ? perm : nullptr, desc_act ? invperm : nullptr, bits,
                         group_size, sym, static_groups, blocksize, qweight, scales, zeros, g_idx, Wk, Err, codesT,

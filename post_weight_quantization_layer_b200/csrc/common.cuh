@@ -82,12 +82,16 @@ int dgemm(cudaStream_t s, int64_t M, int64_t N, int64_t K, double alpha, const d
           const double* B, int64_t ldb, bool transB, double beta, double* C, int64_t ldc, bool upper,
           int tri = 0);
 
-// factor.cu: U (sweep order, fp64) and perm from H.  `work` holds factor_work_bytes(n),
-// `small` factor_small_bytes(n); `status` is a device int.
+// factor.cu: U (sweep order, fp64) and perm from H, stream-ordered on s.  `work` holds
+// factor_work_bytes(n, side != nullptr), `small` factor_small_bytes(n); `status` is a device
+// int.  With a side stream (and two events for its ordering) the top level's T product runs
+// on `side`, concurrently with the left half of the recursion; the call leaves no work on
+// `side` that s does not wait for.
 size_t factor_small_bytes(int64_t n);
-size_t factor_work_bytes(int64_t n);
+size_t factor_work_bytes(int64_t n, bool overlap);
 int factor_hessian(const float* H, int64_t n, float damp, bool desc_act, double* U, int32_t* perm,
-                   int32_t* invperm, void* work, void* small, int* status, cudaStream_t s);
+                   int32_t* invperm, void* work, void* small, int* status, cudaStream_t s,
+                   cudaStream_t side = nullptr, cudaEvent_t ev_p = nullptr, cudaEvent_t ev_t = nullptr);
 
 // sweep.cu: everything after the factor.
 struct SweepArgs {
@@ -120,7 +124,7 @@ enum LanePrio { kLaneHigh = 0, kLaneLow = 1 };
 struct Lane {
   cudaStream_t st = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;
-  cudaEvent_t aux = nullptr;  // free for the leasing call's own ordering
+  cudaEvent_t aux = nullptr, aux2 = nullptr;  // free for the leasing call's own ordering
 };
 class LaneLease {
  public:

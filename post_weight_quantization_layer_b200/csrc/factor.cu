@@ -308,10 +308,11 @@ void plan(int64_t n, int depth, size_t& pmax, std::vector<size_t>& tmax) {
 
 struct Scratch {
   real* P;
+  real* P0;  // the top level's own P when its T product overlaps the left recursion
   std::vector<real*> T;
 };
 
-size_t scratch_elems(int64_t n, Scratch* out, real* base) {
+size_t scratch_elems(int64_t n, Scratch* out, real* base, bool overlap) {
   size_t pmax = 0;
   std::vector<size_t> tmax;
   plan(n, 0, pmax, tmax);
@@ -323,6 +324,8 @@ size_t scratch_elems(int64_t n, Scratch* out, real* base) {
   };
   real* P = take(pmax);
   if (out) out->P = P;
+  real* P0 = (overlap && !tmax.empty()) ? take(tmax[0]) : nullptr;
+  if (out) out->P0 = P0;
   for (size_t d = 0; d < tmax.size(); ++d) {
     real* t = take(tmax[d]);
     if (out) out->T.push_back(t);
@@ -330,27 +333,43 @@ size_t scratch_elems(int64_t n, Scratch* out, real* base) {
   return off;
 }
 
+// Overlap of the top level's T = P U22 with the left recursion: T runs on `side` while the
+// left half (latency-bound leaves and small GEMMs deeper down) runs on the main stream.
+struct Overlap {
+  cudaStream_t side = nullptr;
+  cudaEvent_t p_ready = nullptr, t_ready = nullptr;
+};
+
 // Factor and invert the block [lo, hi) of A (upper triangle valid: the Schur complement
 // with respect to every column right of hi); writes U[lo:hi, lo:hi].
 int factor_rec(real* A, real* R, int64_t n, int64_t lo, int64_t hi, int depth, Scratch& sc, int* status,
-               cudaStream_t s) {
+               cudaStream_t s, const Overlap& ov) {
   const int64_t m = hi - lo;
   if (m <= NB) {
     chol_diag_kernel<<<1, DIAG_THREADS, DIAG_SMEM, s>>>(A, n, lo, static_cast<int>(m), R, status);
     return after_launch();
   }
   const int64_t n2 = right_part(m), n1 = m - n2, mid = hi - n2;
-  GPTQ_TRY(factor_rec(A, R, n, mid, hi, depth + 1, sc, status, s));
+  GPTQ_TRY(factor_rec(A, R, n, mid, hi, depth + 1, sc, status, s, ov));
   real* U22 = R + mid * n + mid;
-  real* P = sc.P;
+  const bool overlap = depth == 0 && ov.side != nullptr && sc.P0 != nullptr;
+  real* P = overlap ? sc.P0 : sc.P;
   real* T = sc.T[depth];
   // P = B U22^T
   GPTQ_TRY(dgemm(s, n1, n2, n2, 1.0, A + lo * n + mid, n, U22, n, true, 0.0, P, n2, false, kTriBTUpper));
   // A' = A - P P^T (upper tiles)
   GPTQ_TRY(dgemm(s, n1, n1, n2, -1.0, P, n2, P, n2, true, 1.0, A + lo * n + lo, n, true));
   // T = P U22
-  GPTQ_TRY(dgemm(s, n1, n2, n2, 1.0, P, n2, U22, n, false, 0.0, T, n2, false, kTriBUpper));
-  GPTQ_TRY(factor_rec(A, R, n, lo, mid, depth + 1, sc, status, s));
+  cudaStream_t st = s;
+  if (overlap) {
+    GPTQ_CUDA(cudaEventRecord(ov.p_ready, s));
+    GPTQ_CUDA(cudaStreamWaitEvent(ov.side, ov.p_ready, 0));
+    st = ov.side;
+  }
+  GPTQ_TRY(dgemm(st, n1, n2, n2, 1.0, P, n2, U22, n, false, 0.0, T, n2, false, kTriBUpper));
+  if (overlap) GPTQ_CUDA(cudaEventRecord(ov.t_ready, ov.side));
+  GPTQ_TRY(factor_rec(A, R, n, lo, mid, depth + 1, sc, status, s, ov));
+  if (overlap) GPTQ_CUDA(cudaStreamWaitEvent(s, ov.t_ready, 0));
   // U12 = -U11 T
   return dgemm(s, n1, n2, n1, -1.0, R + lo * n + lo, n, T, n2, false, 0.0, R + lo * n + mid, n, false, kTriAUpper);
 }
@@ -359,19 +378,22 @@ int factor_rec(real* A, real* R, int64_t n, int64_t lo, int64_t hi, int depth, S
 
 size_t factor_small_bytes(int64_t n) { return 256; }
 
-size_t factor_work_bytes(int64_t n) {
-  return (static_cast<size_t>(n) * n + scratch_elems(n, nullptr, nullptr)) * sizeof(real);
+size_t factor_work_bytes(int64_t n, bool overlap) {
+  return (static_cast<size_t>(n) * n + scratch_elems(n, nullptr, nullptr, overlap)) * sizeof(real);
 }
 
 int factor_hessian(const float* H, int64_t n, float damp, bool desc_act, double* U, int32_t* perm,
-                   int32_t* invperm, void* work, void* small, int* status, cudaStream_t s) {
+                   int32_t* invperm, void* work, void* small, int* status, cudaStream_t s, cudaStream_t side,
+                   cudaEvent_t ev_p, cudaEvent_t ev_t) {
   static cudaError_t attr = cudaFuncSetAttribute(chol_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  DIAG_SMEM);
   if (attr != cudaSuccess) return GPTQ_ERR_CUDA;
   double* dsum = reinterpret_cast<double*>(small);
   real* A = static_cast<real*>(work);  // damped (permuted) Hessian, then Schur complements
   Scratch sc;
-  scratch_elems(n, &sc, A + static_cast<size_t>(n) * n);
+  scratch_elems(n, &sc, A + static_cast<size_t>(n) * n, side != nullptr);
+  Overlap ov;
+  if (side) ov = Overlap{side, ev_p, ev_t};
 
   GPTQ_CUDA(cudaMemsetAsync(dsum, 0, sizeof(double), s));
   diag_sum_kernel<<<std::min<int64_t>((n + 255) / 256, 148), 256, 0, s>>>(H, n, dsum);
@@ -385,7 +407,7 @@ int factor_hessian(const float* H, int64_t n, float damp, bool desc_act, double*
   GPTQ_TRY(after_launch());
   // U starts as zeros: the GEMMs skip its (exactly zero) lower triangle.
   GPTQ_CUDA(cudaMemsetAsync(U, 0, static_cast<size_t>(n) * n * sizeof(real), s));
-  return factor_rec(A, U, n, 0, n, 0, sc, status, s);
+  return factor_rec(A, U, n, 0, n, 0, sc, status, s, ov);
 }
 
 }  // namespace gptq

@@ -26,11 +26,11 @@ int create_lane(LanePrio prio, Lane** out) {
   Lane* l = new Lane;
   bool ok = cudaStreamCreateWithPriority(&l->st, cudaStreamNonBlocking, prio == kLaneHigh ? greatest : least) ==
             cudaSuccess;
-  for (cudaEvent_t* e : {&l->fork, &l->join, &l->aux})
+  for (cudaEvent_t* e : {&l->fork, &l->join, &l->aux, &l->aux2})
     ok = ok && cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess;
   if (!ok) {
     cudaGetLastError();
-    for (cudaEvent_t e : {l->fork, l->join, l->aux})
+    for (cudaEvent_t e : {l->fork, l->join, l->aux, l->aux2})
       if (e) cudaEventDestroy(e);
     if (l->st) cudaStreamDestroy(l->st);
     delete l;

@@ -75,7 +75,7 @@ extern "C" int gptq_factor_hessian_noalloc(const float* H, int64_t n_in, float d
   if (n_in > kNoAllocMaxN) return GPTQ_ERR_UNSUPPORTED;  // beyond the fixed scratch
   if (n_in % 8 != 0) return GPTQ_ERR_UNSUPPORTED;
   if (!aligned16(H) || !aligned16(U) || !aligned16(perm)) return GPTQ_ERR_UNSUPPORTED;
-  if (factor_work_bytes(n_in) > kWorkBytes || factor_small_bytes(n_in) > kSmallBytes) return GPTQ_ERR_UNSUPPORTED;
+  if (factor_work_bytes(n_in, false) > kWorkBytes || factor_small_bytes(n_in) > kSmallBytes) return GPTQ_ERR_UNSUPPORTED;
 
   unsigned char* base = nullptr;
   GPTQ_TRY(scratch_address(&base));

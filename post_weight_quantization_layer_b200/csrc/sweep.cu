@@ -49,7 +49,10 @@ constexpr int EP = KC + 4, UP = PW + 4;  // padded pitches (conflict-free fragme
 // (the accumulated update [ROWS][UP] reuses the U staging buffers)
 constexpr int PANEL_SMEM = PW * PW * 8 + PW * 8 + PW * ROWS * 8 + PW * ROWS + (2 * (ROWS * EP + KC * UP)) * 8;
 static_assert(ROWS * UP <= 2 * KC * UP, "accumulator tile must fit in the staging buffers");
-constexpr int OUTER = 512;             // outer block width (left-looking K stays below it)
+// Outer block width (the left-looking K inside a block stays below it), measured best on
+// this part: 256 for rows of up to 6144 columns, 512 for longer rows (whose trailing GEMMs
+// are large enough to amortise a wider block's panels).
+int outer_block_width(int64_t n_in) { return n_in <= 6144 ? 256 : 512; }
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool pred) {
   const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
@@ -501,7 +504,7 @@ int run_sweep(SweepArgs& a, cudaStream_t s, int* panel_width, int* outer_width) 
   // error has reached the whole group (through the outer update) when its parameters are
   // computed at its first column.
   const int64_t Q = (dynamic_groups && g > P) ? static_cast<int64_t>(g)
-                                              : static_cast<int64_t>(P) * std::max<int64_t>(1, OUTER / P);
+                                              : static_cast<int64_t>(P) * std::max<int64_t>(1, outer_block_width(n_in) / P);
   if (panel_width) *panel_width = P;
   if (outer_width) *outer_width = static_cast<int>(std::min<int64_t>(Q, n_in));
 
