@@ -223,15 +223,6 @@ __global__ void __launch_bounds__(PTHREADS) sweep_panel_kernel(PanelArgs a) {
       pz[c * ROWS + rloc] = active ? a.zeros[g * n_out + row] : 0;
     }
   }
-  // The panel's running weights live in registers in fp64: each column of the panel
-  // receives up to PW-1 compensation updates here, and rounding the running value to
-  // fp32 after each of them would push near-tie codes across a rounding boundary.
-  double v[NCOL];
-#pragma unroll
-  for (int m = 0; m < NCOL; ++m) {
-    const int col = tsub + TPR * m;
-    v[m] = (active && col < pw) ? a.Wk[row * n_in + j0 + col] : 0.0;
-  }
   __syncthreads();
   if (tid < pw) rdiag[tid] = 1.0 / Us[tid * PW + tid];
 
@@ -313,8 +304,18 @@ __global__ void __launch_bounds__(PTHREADS) sweep_panel_kernel(PanelArgs a) {
       Cs[(w * 8 + g) * UP + nb * 8 + 2 * t + 1] = acc[nb][1];
     }
     __syncthreads();
+  }
+  // The panel's running weights live in registers in fp64: each column of the panel
+  // receives up to PW-1 compensation updates here, and rounding the running value to
+  // fp32 after each of them would push near-tie codes across a rounding boundary.  They
+  // are loaded after the left-looking product, so its accumulators and these registers
+  // are never live together.
+  double v[NCOL];
 #pragma unroll
-    for (int m = 0; m < NCOL; ++m) v[m] -= Cs[rloc * UP + tsub + TPR * m];
+  for (int m = 0; m < NCOL; ++m) {
+    const int col = tsub + TPR * m;
+    v[m] = (active && col < pw) ? a.Wk[row * n_in + j0 + col] : 0.0;
+    if (a.j0 > a.o0) v[m] -= Cs[rloc * UP + col];
   }
   __syncthreads();
 
@@ -369,11 +370,13 @@ __global__ void __launch_bounds__(PTHREADS) sweep_panel_kernel(PanelArgs a) {
         cs[c * ROWS + rloc] = static_cast<uint8_t>(q);
         lsum += err * err;
       }
+      // Compensate this thread's later columns.  Only its slot m can hold a column at or
+      // before c (tsub <= o); every later slot is past c.  Columns beyond the panel width
+      // meet zero entries of Us and stay zero.
+      const double* urow = Us + c * PW + tsub;
+      if (tsub > o) v[m] = fma(-err, urow[TPR * m], v[m]);
 #pragma unroll
-      for (int mm = m; mm < NCOL; ++mm) {
-        const int col = tsub + TPR * mm;
-        if (col > c) v[mm] = fma(-err, Us[c * PW + col], v[mm]);
-      }
+      for (int mm = m + 1; mm < NCOL; ++mm) v[mm] = fma(-err, urow[TPR * mm], v[mm]);
     }
   }
 
