@@ -207,7 +207,12 @@ __global__ void __launch_bounds__(PTHREADS) sweep_panel_kernel(PanelArgs a) {
   const unsigned FULL = 0xffffffffu;
   const int base_lane = lane & ~(TPR - 1);
 
-  for (int e = tid; e < PW * PW; e += PTHREADS) {
+  // The panel's block of U (upper triangle): a fixed trip count, fully unrolled, so every
+  // thread's loads are in flight together (each thread reads one column of 32 rows).
+  static_assert((PW * PW) % PTHREADS == 0, "U block staging");
+#pragma unroll
+  for (int i = 0; i < PW * PW / PTHREADS; ++i) {
+    const int e = tid + i * PTHREADS;
     const int r = e / PW, c = e % PW;
     Us[e] = (r < pw && c < pw && c >= r) ? a.U[(j0 + r) * n_in + j0 + c] : 0.0;
   }
@@ -215,12 +220,35 @@ __global__ void __launch_bounds__(PTHREADS) sweep_panel_kernel(PanelArgs a) {
   // than the panel): stage them per column so the serial chain below never waits on
   // global memory.
   if (!a.in_panel_params) {
-    for (int c = tsub; c < pw; c += TPR) {
-      const int64_t j = j0 + c;
-      int64_t g = 0;
-      if (a.gsz > 0) g = (a.static_groups && a.perm) ? clamp_idx(a.perm[j], n_in) / a.gsz : j / a.gsz;
-      ps[c * ROWS + rloc] = active ? a.scales[g * n_out + row] : 1.f;
-      pz[c * ROWS + rloc] = active ? a.zeros[g * n_out + row] : 0;
+    // Three phases, each with all of a thread's loads in flight together: group indices,
+    // then the parameters (read-only path), then the shared-memory stores.  32-bit index
+    // arithmetic (n_in < 2^16).
+    int gi[NCOL];
+    const int nin = static_cast<int>(n_in), jj0 = static_cast<int>(j0);
+#pragma unroll
+    for (int m = 0; m < NCOL; ++m) {
+      const int c = tsub + TPR * m;
+      const int j = jj0 + c;
+      int col = j;
+      if (a.static_groups && a.perm && c < pw) col = min(max(__ldg(a.perm + j), 0), nin - 1);
+      gi[m] = (a.gsz > 0 && c < pw) ? col / a.gsz : 0;
+    }
+    float sv[NCOL];
+    int zv[NCOL];
+#pragma unroll
+    for (int m = 0; m < NCOL; ++m) {
+      const int64_t at = static_cast<int64_t>(gi[m]) * n_out + row;
+      const bool ld = active && tsub + TPR * m < pw;
+      sv[m] = ld ? __ldg(a.scales + at) : 1.f;
+      zv[m] = ld ? __ldg(a.zeros + at) : 0;
+    }
+#pragma unroll
+    for (int m = 0; m < NCOL; ++m) {
+      const int c = tsub + TPR * m;
+      if (c < pw) {
+        ps[c * ROWS + rloc] = sv[m];
+        pz[c * ROWS + rloc] = zv[m];
+      }
     }
   }
   __syncthreads();
@@ -332,7 +360,7 @@ __global__ void __launch_bounds__(PTHREADS) sweep_panel_kernel(PanelArgs a) {
     for (int o = 0; o < TPR; ++o) {
       const int c = m * TPR + o;
       if (c >= pw) break;
-      const int64_t j = j0 + c;
+      const int j = static_cast<int>(j0) + c;  // < 2^16: 32-bit division below
       if (a.in_panel_params && j % a.gsz == 0) {
         float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
@@ -351,8 +379,8 @@ __global__ void __launch_bounds__(PTHREADS) sweep_panel_kernel(PanelArgs a) {
         }
         group_params(mn, mx, a.bits, a.sym != 0, s, z);
         if (tsub == 0 && active) {
-          a.scales[(j / a.gsz) * n_out + row] = s;
-          a.zeros[(j / a.gsz) * n_out + row] = z;
+          a.scales[static_cast<int64_t>(j / a.gsz) * n_out + row] = s;
+          a.zeros[static_cast<int64_t>(j / a.gsz) * n_out + row] = z;
         }
       }
       // All threads of the row take the decision on the owner's current value, so the
