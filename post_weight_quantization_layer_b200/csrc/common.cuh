@@ -64,17 +64,10 @@ constexpr int kStatusTimeout = GPTQ_ERR_TIMEOUT;
 int launch_hessian(const void* X, int x_dtype, int64_t tokens, int64_t n, float* H, cudaStream_t s);
 int hessian_device_status(cudaStream_t s, int clear);
 
-// gemm.cu: C[m,n] = beta*C[m,n] + alpha * sum_k A[m*lda+k] * B(k,n),
-// B(k,n) = transB ? B[n*ldb+k] : B[k*ldb+n].  upper != 0 skips 128x128 tiles of C
-// lying entirely below its diagonal (m > n for every element).
-int sgemm(cudaStream_t s, int64_t M, int64_t N, int64_t K, float alpha, const float* A, int64_t lda,
-          const float* B, int64_t ldb, bool transB, float beta, float* C, int64_t ldc, bool upper);
-// Same product (fp32 operands, fp32 accumulation) applied to an fp64 C:
-// C[m,n] = C[m,n] + (double)(alpha * sum_k A[m,k] B(k,n)).
-int sgemm_acc64(cudaStream_t s, int64_t M, int64_t N, int64_t K, float alpha, const float* A, int64_t lda,
-                const float* B, int64_t ldb, double* C, int64_t ldc);
-// fp64 operands, fp64 accumulation (same conventions as sgemm).  `tri` declares operands
-// that are triangular with exact zeros elsewhere, so that those K ranges are skipped:
+// gemm.cu: fp64 C[m,n] = beta*C[m,n] + alpha * sum_k A[m*lda+k] * B(k,n),
+// B(k,n) = transB ? B[n*ldb+k] : B[k*ldb+n].  upper != 0 skips tiles of C lying entirely
+// below its diagonal (m > n for every element).  `tri` declares operands that are
+// triangular with exact zeros elsewhere, so that those K ranges are skipped:
 constexpr int kTriAUpper = 1;   // A(m,k) == 0 for k < m
 constexpr int kTriBUpper = 2;   // B(k,n) == 0 for k > n   (op(B) upper triangular)
 constexpr int kTriBTUpper = 4;  // B(k,n) == 0 for k < n   (op(B) = U^T with U upper)

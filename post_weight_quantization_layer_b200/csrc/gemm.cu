@@ -1,13 +1,11 @@
-// GEMM on the CUDA cores in fp32 (lazy block updates of the sweep) and fp64 (rank-k
-// updates of the factorisation): C = beta*C + alpha * A * op(B).
+// fp64 GEMMs of the factorisation (its rank-k updates) and of the sweep (its lazy block
+// updates): C = beta*C + alpha * A * op(B).
 //
-// 128x128 tile per 256-thread CTA, 8x8 outputs per thread, K staged 8 at a time through
-// double-buffered shared memory.  All operands are row-major with arbitrary leading
-// dimensions; every global access is bounds-checked, so ragged edges need no padding.
-//
-// In-place use: when C aliases A (or B) the call is still correct as long as each CTA
-// is the only reader of the A rows (B columns) it writes, i.e. N <= 128 (M <= 128),
-// because a CTA reads all of K before its epilogue writes.  The callers rely on this.
+// Two kernels.  dgemm_mma_kernel (below) runs on the fp64 matrix units and takes every
+// call whose operands are 16-byte aligned with even leading dimensions, K and N.
+// gemm_kernel is the CUDA-core fallback for the rest: 128x128 tile per 256-thread CTA,
+// 8x8 outputs per thread, K staged 8 at a time through double-buffered shared memory,
+// every global access bounds-checked, so ragged edges need no padding.
 #include "common.cuh"
 
 namespace gptq {
@@ -275,18 +273,6 @@ __global__ void __maxnreg__(192) dgemm_mma_kernel(int64_t M, int64_t N, int64_t 
 
 }  // namespace
 
-int sgemm(cudaStream_t s, int64_t M, int64_t N, int64_t K, float alpha, const float* A, int64_t lda,
-          const float* B, int64_t ldb, bool transB, float beta, float* C, int64_t ldc, bool upper) {
-  if (M <= 0 || N <= 0) return GPTQ_OK;
-  dim3 grid(static_cast<unsigned>((N + TN - 1) / TN), static_cast<unsigned>((M + TM - 1) / TM));
-  if (grid.y > 65535u) return GPTQ_ERR_UNSUPPORTED;
-  if (transB)
-    gemm_kernel<float, true, float><<<grid, 256, 0, s>>>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc, upper ? 1 : 0, 0);
-  else
-    gemm_kernel<float, false, float><<<grid, 256, 0, s>>>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc, upper ? 1 : 0, 0);
-  return after_launch();
-}
-
 int dgemm(cudaStream_t s, int64_t M, int64_t N, int64_t K, double alpha, const double* A, int64_t lda,
           const double* B, int64_t ldb, bool transB, double beta, double* C, int64_t ldc, bool upper, int tri) {
   if (M <= 0 || N <= 0) return GPTQ_OK;
@@ -356,13 +342,5 @@ int dgemm(cudaStream_t s, int64_t M, int64_t N, int64_t K, double alpha, const d
   return after_launch();
 }
 
-int sgemm_acc64(cudaStream_t s, int64_t M, int64_t N, int64_t K, float alpha, const float* A, int64_t lda,
-                const float* B, int64_t ldb, double* C, int64_t ldc) {
-  if (M <= 0 || N <= 0) return GPTQ_OK;
-  dim3 grid(static_cast<unsigned>((N + TN - 1) / TN), static_cast<unsigned>((M + TM - 1) / TM));
-  if (grid.y > 65535u) return GPTQ_ERR_UNSUPPORTED;
-  gemm_kernel<float, false, double><<<grid, 256, 0, s>>>(M, N, K, alpha, A, lda, B, ldb, 1.f, C, ldc, 0, 0);
-  return after_launch();
-}
 
 }  // namespace gptq

@@ -14,8 +14,9 @@
 // * codesT [n_in, n_out] uint8 holds the codes in sweep order (column-major w.r.t. W),
 //   so both the sweep's writes and the packer's reads are coalesced across rows.
 // * Panels of P <= 64 columns: one kernel per panel, rows in parallel (4 threads per row,
-//   16 columns per thread in registers, the panel's block of U in shared memory, group
-//   min/max and the error broadcast via warp shuffles).
+//   16 columns per thread in registers, the panel's block of U in shared memory; per
+//   column the owner's current value goes to the row's threads by one warp shuffle and
+//   all of them take the decision; group min/max by warp shuffles).
 // * Precision: the running weights, the errors, U and the lazy-update products are all
 //   fp64; only the code decision (w / s, rounding) is taken in fp32.  GPTQ's sweep is a
 //   long chain of rounding decisions, each depending on every earlier error of its row,
@@ -29,7 +30,9 @@
 //   first, on a high-priority stream that then runs the next block's panels; the rest of
 //   the trailing update runs at the same time on a low-priority stream.  The panel chain
 //   (latency-bound, one CTA of 4 warps per SM) shares the SMs with the GEMM's tiles
-//   (one CTA per SM), so the panels' time hides under the matrix-unit work.
+//   (one CTA per SM), so the two overlap; where a panel shares its SM with a GEMM CTA its
+//   fp64 instructions wait behind the GEMM's on the shared fp64 pipe, and the panel
+//   chain remains the longer of the two.
 #include <algorithm>
 
 #include "common.cuh"
