@@ -53,3 +53,17 @@ def test_reference_arm_two_ranks_prints_one_line():
     assert len(lines) == 1
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["unit"] == "weight-cols/s" and d["value"] > 0
+
+
+def test_hessian_traffic_profile_parses_per_launch():
+    """The bench's roofline takes the Hessian's DRAM traffic per launch from the committed
+    ncu summary: one figure per distinct Hessian of the Llama-2-7B layer, in launch order,
+    each at least the launch's algorithmic bytes (X once + H once)."""
+    import bench
+    from post_weight_quantization_layer_b200 import synth
+
+    cfg = synth.CONFIGS["llama7b"]
+    traffic = bench.load_traffic()
+    assert traffic is not None and len(traffic) == len(cfg.hessian_n)
+    for n, t in zip(cfg.hessian_n, traffic):
+        assert t >= cfg.tokens * n * 2 + n * n * 4
