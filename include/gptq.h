@@ -8,7 +8,15 @@
  *   current CUDA device.  The library never frees or retains a caller
  *   pointer.  Device pointers must be 16-byte aligned.
  * - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
- *   Work is enqueued on that stream in order.
+ *   Work is enqueued on that stream in order.  Some calls also run work on
+ *   library-owned streams forked from `stream`; all of it is joined back into
+ *   `stream` before the call returns, so callers see one stream-ordered call.
+ * - Calls from several host threads may run at once: each leases its own
+ *   library streams and workspace.  Exceptions: gptq_factor_hessian_noalloc
+ *   (one shared scratch array), and gptq_device_status, which reports a
+ *   timeout recorded by any call on the device since it was last cleared.
+ * - One process per GPU: the kernels' shared-memory limits are configured for
+ *   the device that is current at a process's first call.
  * - The return value is a gptq_status.  Arguments are validated on the host
  *   before any work is enqueued; a rejected call changes no output.
  * - Notation: W is [n_out, n_in] (a torch.nn.Linear weight), X is

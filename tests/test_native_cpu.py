@@ -117,3 +117,4 @@ def test_python_binding_fails_loudly_without_cuda_tensors():
     import post_weight_quantization_layer_b200 as gq
     with pytest.raises(ValueError):
         gq.quantize_layer(torch.zeros(4, 8), torch.zeros(8, 8))
+
