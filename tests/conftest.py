@@ -20,6 +20,15 @@ def golden_dir():
     return GOLDEN
 
 
+@pytest.fixture(scope="session", autouse=True)
+def _native_library_built(request):
+    """When GPU tests are selected, compile the native library once per session if it is
+    missing or older than its sources (a fresh checkout carries no built library)."""
+    if any(item.get_closest_marker("gpu") for item in request.session.items):
+        from post_weight_quantization_layer_b200.build import build
+        build(force=False)
+
+
 def read_golden(name):
     """Non-comment, non-empty lines of a golden fixture."""
     with open(os.path.join(GOLDEN, name)) as f:
