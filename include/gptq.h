@@ -15,8 +15,9 @@
  *   library streams and workspace.  Exceptions: gptq_factor_hessian_noalloc
  *   (one shared scratch array), and gptq_device_status, which reports a
  *   timeout recorded by any call on the device since it was last cleared.
- * - One process per GPU: the kernels' shared-memory limits are configured for
- *   the device that is current at a process's first call.
+ * - One process may drive several GPUs: per-device state (kernel shared-memory
+ *   limits, workspace pool, library streams, the no-alloc scratch address) is set up
+ *   on first use on each device, for the device that is current at the call.
  * - The return value is a gptq_status.  Arguments are validated on the host
  *   before any work is enqueued; a rejected call changes no output.
  * - Notation: W is [n_out, n_in] (a torch.nn.Linear weight), X is
@@ -77,6 +78,11 @@ typedef struct {
  *         tokens accumulate (streaming calibration).  Products are exact in
  *         fp32; sums are fp32 with periodic re-normalisation of the
  *         tensor-core accumulator (relative Frobenius error <= 1e-5).
+ *         Not bitwise reproducible: the partial sums of different token
+ *         segments are added into H with fp32 atomics, whose order varies from
+ *         run to run, so two runs may differ in the last bits of H (and codes
+ *         computed from H may then differ near rounding ties).  Everything after
+ *         H (factor, sweep, packing) is deterministic for a given H.
  * Asynchronous on `stream`: only host-detectable errors are returned.  A
  * device-side timeout is recorded and reported by gptq_device_status().
  */
@@ -188,7 +194,8 @@ int gptq_quantize_layer_factored(const void* W, int w_dtype, int64_t n_out, int6
  * someone else - an inference or serving runtime that reserves a fixed arena at
  * start-up, a real-time loop that must not call an allocator, a plugin whose host caps
  * the allocator.  gptq_factor_hessian takes its workspace from a memory pool; this
- * variant runs the same kernels with the same arguments, outputs and results, but its
+ * variant runs the same kernels with the same arguments and outputs, and gives the same
+ * results bit for bit (the factor's kernels are deterministic), but its
  * scratch is one fixed array of device memory built into the library (about 13.3 MB,
  * held on every GPU that loads the library until the process exits).  It calls no
  * cudaMalloc, cudaFree or other allocating routine.
@@ -197,6 +204,13 @@ int gptq_quantize_layer_factored(const void* W, int w_dtype, int64_t n_out, int6
  * - n_in <= 1024 (and a multiple of 8); larger sizes return GPTQ_ERR_UNSUPPORTED.
  * - The first call on a device looks up the array's device address on that device
  *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ * - When the array is placed on the GPU: the array is part of the library's device code,
+ *   and it occupies device memory from the moment that code is loaded on a device.  Under
+ *   CUDA's lazy module loading (the default of CUDA 12) that happens inside the first call
+ *   of this function on that device, so the FIRST call does take about 13.3 MB of device
+ *   memory, and fails with GPTQ_ERR_CUDA if none is left.  A caller that reserves a fixed
+ *   arena makes one call (or runs with CUDA_MODULE_LOADING=EAGER) before reserving it;
+ *   every later call allocates nothing.
  * - All calls share the one array and it keeps the last call's contents; calls that
  *   may overlap on the GPU (different streams, different host threads) race and must be
  *   serialised by the caller.

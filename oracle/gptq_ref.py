@@ -18,7 +18,7 @@ describe:
 Where a floating-point value decides an integer code, the decision is taken in
 float32, the precision the GPU kernels use; every other step is float64.
 
-Readings taken where the pages are silent (each also listed in the design doc):
+Readings taken where the pages are silent:
 * rounding is round-half-to-even; division is IEEE x / s, never x * (1/s);
 * sym: s = 2*max|x| / maxq, zero = 2^(bits-1);
 * asym: range [min(0, min x), max(0, max x)], s = (hi-lo)/maxq, zero = rint(-lo/s);

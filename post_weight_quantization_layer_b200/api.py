@@ -41,11 +41,35 @@ def _ptr(t):
 
 
 def _need_cuda(*ts):
+    """Every tensor must be a contiguous CUDA tensor on the current device (checked last, so
+    that shape and dtype errors are reported first)."""
     for t in ts:
-        if not (isinstance(t, torch.Tensor) and t.is_cuda):
-            raise ValueError("tensors must be CUDA tensors")
+        if not isinstance(t, torch.Tensor):
+            raise ValueError("arguments must be torch tensors")
         if not t.is_contiguous():
             raise ValueError("tensors must be contiguous")
+        if not t.is_cuda:
+            raise ValueError("tensors must be CUDA tensors")
+        if t.device.index != torch.cuda.current_device():
+            raise ValueError(f"tensor on {t.device}, but the current device is cuda:{torch.cuda.current_device()}")
+
+
+def _need(t, what, dtypes, shape):
+    """Shape and dtype of one argument (raises ValueError before any native call)."""
+    if not isinstance(t, torch.Tensor):
+        raise ValueError(f"{what} must be a torch tensor")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{what} must have dtype {' or '.join(str(d) for d in dtypes)}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{what} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _weight(W):
+    if not isinstance(W, torch.Tensor) or W.dim() != 2:
+        raise ValueError("W must be a 2-D [n_out, n_in] tensor")
+    if W.dtype not in _DTYPE:
+        raise ValueError(f"W must be float32, float16 or bfloat16, got {W.dtype}")
+    return W.shape
 
 
 def group_count(n_in: int, group_size: int) -> int:
@@ -63,9 +87,11 @@ class QuantResult:
 
 def accumulate_hessian(X: torch.Tensor, H: torch.Tensor, stream=None) -> torch.Tensor:
     """H += 2 X^T X (asynchronous on the stream).  X [T, n] fp16/bf16, H [n, n] fp32."""
+    if not isinstance(X, torch.Tensor) or X.dim() != 2:
+        raise ValueError("X must be a 2-D [tokens, n_in] tensor")
+    _need(X, "X", (torch.float16, torch.bfloat16), tuple(X.shape))
+    _need(H, "H", (torch.float32,), (X.shape[1], X.shape[1]))
     _need_cuda(X, H)
-    if X.dim() != 2 or H.shape != (X.shape[1], X.shape[1]) or H.dtype != torch.float32:
-        raise ValueError("X must be [tokens, n_in] and H [n_in, n_in] float32")
     st = lib().gptq_accumulate_hessian(_ptr(X), _DTYPE.get(X.dtype, 99), X.shape[0], X.shape[1], _ptr(H),
                                        _stream(stream))
     _check(st, "gptq_accumulate_hessian")
@@ -81,13 +107,25 @@ def launch_count() -> int:
 
 
 def _outputs(n_out, n_in, bits, group_size, device, out):
-    if out is not None:
-        return out
-    G = group_count(n_in, group_size)
-    return (torch.empty(n_in * bits // 32, n_out, dtype=torch.int32, device=device),
-            torch.empty(G, n_out, dtype=torch.float32, device=device),
-            torch.empty(G, n_out, dtype=torch.int32, device=device),
-            torch.empty(n_in, dtype=torch.int32, device=device))
+    """Output tensors (qweight, scales, zeros, g_idx): allocated here, or the caller's
+    `out` tuple after checking that every piece has the shape and dtype the call writes."""
+    # an invalid group size is rejected by the native call, which then writes nothing
+    G = group_count(n_in, group_size) if (group_size == -1 or group_size > 0) else 1
+    words = n_in * bits // 32
+    if out is None:
+        return (torch.empty(words, n_out, dtype=torch.int32, device=device),
+                torch.empty(G, n_out, dtype=torch.float32, device=device),
+                torch.empty(G, n_out, dtype=torch.int32, device=device),
+                torch.empty(n_in, dtype=torch.int32, device=device))
+    if not isinstance(out, (tuple, list)) or len(out) != 4:
+        raise ValueError("out must be a tuple (qweight, scales, zeros, g_idx)")
+    qw, sc, zr, gi = out
+    _need(qw, "out qweight", (torch.int32,), (words, n_out))
+    _need(sc, "out scales", (torch.float32,), (G, n_out))
+    _need(zr, "out zeros", (torch.int32,), (G, n_out))
+    _need(gi, "out g_idx", (torch.int32,), (n_in,))
+    _need_cuda(qw, sc, zr, gi)
+    return tuple(out)
 
 
 def _stats_dict(s: GptqStats):
@@ -97,9 +135,10 @@ def _stats_dict(s: GptqStats):
 def quantize_layer(W, H, bits=4, group_size=128, damp_percent=0.01, sym=True, desc_act=False,
                    static_groups=False, blocksize=128, stats=False, out=None, stream=None) -> QuantResult:
     """GPTQ of one linear layer: W [n_out, n_in] (fp32/fp16/bf16), H [n_in, n_in] fp32."""
-    _need_cuda(W, H)
-    n_out, n_in = W.shape
+    n_out, n_in = _weight(W)
+    _need(H, "H", (torch.float32,), (n_in, n_in))
     qw, sc, zr, gi = _outputs(n_out, n_in, bits, group_size, W.device, out)
+    _need_cuda(W, H)
     st_obj = GptqStats() if stats else None
     st = lib().gptq_quantize_layer(
         _ptr(W), _DTYPE.get(W.dtype, 99), n_out, n_in, _ptr(H), bits, group_size, float(damp_percent),
@@ -111,8 +150,11 @@ def quantize_layer(W, H, bits=4, group_size=128, damp_percent=0.01, sym=True, de
 
 def factor_hessian(H, damp_percent=0.01, desc_act=False, stream=None):
     """Returns (U, perm): inverse(H_d) = U^T U in sweep order (fp64), perm = column order."""
-    _need_cuda(H)
+    if not isinstance(H, torch.Tensor) or H.dim() != 2:
+        raise ValueError("H must be a square 2-D tensor")
     n = H.shape[0]
+    _need(H, "H", (torch.float32,), (n, n))
+    _need_cuda(H)
     U = torch.empty(n, n, dtype=torch.float64, device=H.device)
     perm = torch.empty(n, dtype=torch.int32, device=H.device)
     st = lib().gptq_factor_hessian(_ptr(H), n, float(damp_percent), int(bool(desc_act)), _ptr(U), _ptr(perm),
@@ -126,6 +168,12 @@ def factor_hessians(Hs, damp_percent=0.01, desc_act=False, stream=None):
     the library).  Returns [(U, perm), ...] in the order of Hs; raises GPTQError naming
     the first item that failed."""
     Hs = list(Hs)
+    if not Hs:
+        raise ValueError("factor_hessians needs at least one Hessian")
+    for i, H in enumerate(Hs):
+        if not isinstance(H, torch.Tensor) or H.dim() != 2:
+            raise ValueError(f"H[{i}] must be a square 2-D tensor")
+        _need(H, f"H[{i}]", (torch.float32,), (H.shape[0], H.shape[0]))
     _need_cuda(*Hs)
     k = len(Hs)
     outs = [(torch.empty(H.shape[0], H.shape[0], dtype=torch.float64, device=H.device),
@@ -144,11 +192,11 @@ def factor_hessians(Hs, damp_percent=0.01, desc_act=False, stream=None):
 
 def quantize_layer_factored(W, U, perm, bits=4, group_size=128, sym=True, static_groups=False, blocksize=128,
                             stats=False, out=None, stream=None) -> QuantResult:
-    _need_cuda(W, U, perm)
-    if U.dtype != torch.float64 or perm.dtype != torch.int32:
-        raise ValueError("U must be float64 and perm int32")
-    n_out, n_in = W.shape
+    n_out, n_in = _weight(W)
+    _need(U, "U", (torch.float64,), (n_in, n_in))
+    _need(perm, "perm", (torch.int32,), (n_in,))
     qw, sc, zr, gi = _outputs(n_out, n_in, bits, group_size, W.device, out)
+    _need_cuda(W, U, perm)
     st_obj = GptqStats() if stats else None
     st = lib().gptq_quantize_layer_factored(
         _ptr(W), _DTYPE.get(W.dtype, 99), n_out, n_in, _ptr(U), _ptr(perm), bits, group_size, int(bool(sym)),

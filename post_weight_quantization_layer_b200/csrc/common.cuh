@@ -37,6 +37,11 @@ inline int after_launch() {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Raise a kernel's dynamic shared-memory limit to `bytes` on the current device.  The
+// attribute is per device, so it is set once for every (device, kernel) pair this process
+// launches on; a process may drive several GPUs.  Thread-safe.
+int ensure_smem_limit(const void* kernel, int bytes);
+
 inline int num_sms() {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

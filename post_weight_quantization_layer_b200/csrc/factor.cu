@@ -41,18 +41,21 @@ constexpr int SP = NB + 4;      // pitch of the diagonal block in shared memory 
 constexpr int TP = NB / 2 + 4;  // of m8n8k4 hit 16 distinct bank pairs when pitch = 4 mod 16)
 using real = double;     // working precision of the factorisation
 
-// Sum of diag(H) in double.
-__global__ void diag_sum_kernel(const float* __restrict__ H, int64_t n, double* out) {
+// Sum of diag(H) in double, by one CTA of DSUM_THREADS threads in a fixed order (no
+// atomics), so that the damping term, and with it the whole factor, is the same bit for
+// bit on every call.  At most 65,535 / 1,024 = 64 strided loads a thread.
+constexpr int DSUM_THREADS = 1024;
+__global__ void __launch_bounds__(DSUM_THREADS) diag_sum_kernel(const float* __restrict__ H, int64_t n, double* out) {
   double s = 0.0;
-  for (int64_t i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) s += H[i * n + i];
+  for (int64_t i = threadIdx.x; i < n; i += DSUM_THREADS) s += H[i * n + i];
   for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  __shared__ double ws[32];
+  __shared__ double ws[DSUM_THREADS / 32];
   if ((threadIdx.x & 31) == 0) ws[threadIdx.x >> 5] = s;
   __syncthreads();
   if (threadIdx.x < 32) {
-    s = (threadIdx.x < (blockDim.x >> 5)) ? ws[threadIdx.x] : 0.0;
+    s = ws[threadIdx.x];
     for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (threadIdx.x == 0) atomicAdd(out, s);
+    if (threadIdx.x == 0) *out = s;
   }
 }
 
@@ -385,9 +388,7 @@ size_t factor_work_bytes(int64_t n, bool overlap) {
 int factor_hessian(const float* H, int64_t n, float damp, bool desc_act, double* U, int32_t* perm,
                    int32_t* invperm, void* work, void* small, int* status, cudaStream_t s, cudaStream_t side,
                    cudaEvent_t ev_p, cudaEvent_t ev_t) {
-  static cudaError_t attr = cudaFuncSetAttribute(chol_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 DIAG_SMEM);
-  if (attr != cudaSuccess) return GPTQ_ERR_CUDA;
+  GPTQ_TRY(ensure_smem_limit(reinterpret_cast<const void*>(chol_diag_kernel), DIAG_SMEM));
   double* dsum = reinterpret_cast<double*>(small);
   real* A = static_cast<real*>(work);  // damped (permuted) Hessian, then Schur complements
   Scratch sc;
@@ -395,8 +396,7 @@ int factor_hessian(const float* H, int64_t n, float damp, bool desc_act, double*
   Overlap ov;
   if (side) ov = Overlap{side, ev_p, ev_t};
 
-  GPTQ_CUDA(cudaMemsetAsync(dsum, 0, sizeof(double), s));
-  diag_sum_kernel<<<std::min<int64_t>((n + 255) / 256, 148), 256, 0, s>>>(H, n, dsum);
+  diag_sum_kernel<<<1, DSUM_THREADS, 0, s>>>(H, n, dsum);
   GPTQ_TRY(after_launch());
   if (desc_act) {
     act_order_rank_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(H, n, perm, invperm);

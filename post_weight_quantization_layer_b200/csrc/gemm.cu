@@ -281,25 +281,12 @@ int dgemm(cudaStream_t s, int64_t M, int64_t N, int64_t K, double alpha, const d
   const bool mma_ok = aligned16(A) && aligned16(B) && aligned16(C) && lda % 2 == 0 && ldb % 2 == 0 && ldc % 2 == 0 &&
                       K % 2 == 0 && N % 2 == 0;
   if (mma_ok) {
-    static cudaError_t attr = [] {
-      cudaError_t e[6] = {
-          cudaFuncSetAttribute(dgemm_mma_kernel<true, 128, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               DTile<128, 128>::SMEM),
-          cudaFuncSetAttribute(dgemm_mma_kernel<false, 128, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               DTile<128, 128>::SMEM),
-          cudaFuncSetAttribute(dgemm_mma_kernel<true, 64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               DTile<64, 64>::SMEM),
-          cudaFuncSetAttribute(dgemm_mma_kernel<false, 64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               DTile<64, 64>::SMEM),
-          cudaFuncSetAttribute(dgemm_mma_kernel<true, 32, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               DTile<32, 32>::SMEM),
-          cudaFuncSetAttribute(dgemm_mma_kernel<false, 32, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               DTile<32, 32>::SMEM)};
-      for (cudaError_t x : e)
-        if (x != cudaSuccess) return x;
-      return cudaSuccess;
-    }();
-    if (attr != cudaSuccess) return GPTQ_ERR_CUDA;
+    GPTQ_TRY(ensure_smem_limit(reinterpret_cast<const void*>(dgemm_mma_kernel<true, 128, 128>), DTile<128, 128>::SMEM));
+    GPTQ_TRY(ensure_smem_limit(reinterpret_cast<const void*>(dgemm_mma_kernel<false, 128, 128>), DTile<128, 128>::SMEM));
+    GPTQ_TRY(ensure_smem_limit(reinterpret_cast<const void*>(dgemm_mma_kernel<true, 64, 64>), DTile<64, 64>::SMEM));
+    GPTQ_TRY(ensure_smem_limit(reinterpret_cast<const void*>(dgemm_mma_kernel<false, 64, 64>), DTile<64, 64>::SMEM));
+    GPTQ_TRY(ensure_smem_limit(reinterpret_cast<const void*>(dgemm_mma_kernel<true, 32, 32>), DTile<32, 32>::SMEM));
+    GPTQ_TRY(ensure_smem_limit(reinterpret_cast<const void*>(dgemm_mma_kernel<false, 32, 32>), DTile<32, 32>::SMEM));
     // Small products: 64x64 (or 32x32) tiles spread the work over 4x (16x) more SMs.
     const int64_t big_tiles = ((M + 127) / 128) * ((N + 127) / 128);
     const int64_t mid_tiles = ((M + 63) / 64) * ((N + 63) / 64);

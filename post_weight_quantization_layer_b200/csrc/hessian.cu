@@ -317,12 +317,7 @@ template <uint32_t F>
 int launch_impl(const void* X, int64_t T, int n, float* H, cudaStream_t st) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return GPTQ_ERR_CUDA;
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(hessian_syrk_kernel<F>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-  });
-  if (attr_err != cudaSuccess) return GPTQ_ERR_CUDA;
+  GPTQ_TRY(ensure_smem_limit(reinterpret_cast<const void*>(hessian_syrk_kernel<F>), SMEM_BYTES));
   const int tiles = hsched::tile_count(n);
   const int sms = num_sms();
   // TMA coordinates are 32-bit: walk very long token streams in chunks.

@@ -10,6 +10,7 @@
 // workspace on the caller's stream never overtake a lane.
 #include <map>
 #include <mutex>
+#include <set>
 #include <vector>
 
 #include "common.cuh"
@@ -68,6 +69,24 @@ int LaneLease::acquire(int count, const LanePrio* prio) {
     GPTQ_CUDA(cudaEventRecord(l->fork, s_));
     GPTQ_CUDA(cudaStreamWaitEvent(l->st, l->fork, 0));
   }
+  return GPTQ_OK;
+}
+
+namespace {
+std::mutex g_attr_mu;
+std::set<std::pair<int, const void*>> g_attr_done;  // (device, kernel) pairs already raised
+}  // namespace
+
+int ensure_smem_limit(const void* kernel, int bytes) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GPTQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_attr_mu);
+  if (g_attr_done.count({dev, kernel})) return GPTQ_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    return GPTQ_ERR_CUDA;
+  }
+  g_attr_done.insert({dev, kernel});
   return GPTQ_OK;
 }
 

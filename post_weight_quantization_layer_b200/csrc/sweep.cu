@@ -511,9 +511,7 @@ int stage_and_fixed(const SweepArgs& a, cudaStream_t s) {
 }  // namespace
 
 int run_sweep(SweepArgs& a, cudaStream_t s, int* panel_width, int* outer_width) {
-  static cudaError_t attr =
-      cudaFuncSetAttribute(sweep_panel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PANEL_SMEM);
-  if (attr != cudaSuccess) return GPTQ_ERR_CUDA;
+  GPTQ_TRY(ensure_smem_limit(reinterpret_cast<const void*>(sweep_panel_kernel), PANEL_SMEM));
   const int64_t n_out = a.n_out, n_in = a.n_in;
   const int g = a.group_size;
   const bool dynamic_groups = g > 0 && !a.static_groups;

@@ -118,3 +118,46 @@ def test_python_binding_fails_loudly_without_cuda_tensors():
     with pytest.raises(ValueError):
         gq.quantize_layer(torch.zeros(4, 8), torch.zeros(8, 8))
 
+
+
+def test_python_binding_rejects_mismatched_tensors():
+    """Every wrapper checks dtype, shape and layout of its tensors (and of `out=`) before
+    the native call, so a mismatched tensor can never reach a kernel as a raw pointer."""
+    import torch
+
+    import post_weight_quantization_layer_b200 as gq
+    W = torch.zeros(4, 64)
+    H = torch.zeros(64, 64)
+    cases = [
+        (lambda: gq.quantize_layer(W, H.half()), "H must have dtype"),
+        (lambda: gq.quantize_layer(W, torch.zeros(64, 32)), "H must have shape"),
+        (lambda: gq.quantize_layer(W.int(), H), "W must be float32"),
+        (lambda: gq.quantize_layer(torch.zeros(64), H), "2-D"),
+        (lambda: gq.quantize_layer(W.t(), torch.zeros(4, 4)), "contiguous"),
+        (lambda: gq.quantize_layer(W, H, 4, 32, out=(1, 2, 3)), "out must be a tuple"),
+        (lambda: gq.quantize_layer(W, H, 4, 32, out=(torch.zeros(4, 8, dtype=torch.int32),
+                                                     torch.zeros(2, 4), torch.zeros(2, 4, dtype=torch.int32),
+                                                     torch.zeros(64, dtype=torch.int32))), "out qweight"),
+        (lambda: gq.quantize_layer(W, H, 4, 32, out=(torch.zeros(8, 4, dtype=torch.int32),
+                                                     torch.zeros(1, 4), torch.zeros(2, 4, dtype=torch.int32),
+                                                     torch.zeros(64, dtype=torch.int32))), "out scales"),
+        (lambda: gq.quantize_layer(W, H, 4, 32, out=(torch.zeros(8, 4, dtype=torch.int32),
+                                                     torch.zeros(2, 4), torch.zeros(2, 4),
+                                                     torch.zeros(64, dtype=torch.int32))), "out zeros"),
+        (lambda: gq.factor_hessian(torch.zeros(64, 32)), "H must have shape"),
+        (lambda: gq.factor_hessian(H.double()), "H must have dtype"),
+        (lambda: gq.factor_hessians([]), "at least one"),
+        (lambda: gq.factor_hessians([H, H.half()]), r"H\[1\] must have dtype"),
+        (lambda: gq.quantize_layer_factored(W, H, torch.zeros(64, dtype=torch.int32)), "U must have dtype"),
+        (lambda: gq.quantize_layer_factored(W, H.double()[:32], torch.zeros(64, dtype=torch.int32)),
+         "U must have shape"),
+        (lambda: gq.quantize_layer_factored(W, H.double(), torch.zeros(64, dtype=torch.int64)), "perm must have dtype"),
+        (lambda: gq.quantize_layer_factored(W, H.double(), torch.zeros(60, dtype=torch.int32)), "perm must have shape"),
+        (lambda: gq.accumulate_hessian(torch.zeros(16, 64), H), "X must have dtype"),
+        (lambda: gq.accumulate_hessian(torch.zeros(16, 64, dtype=torch.bfloat16), torch.zeros(32, 32)),
+         "H must have shape"),
+        (lambda: gq.quantize_layer(W, H), "CUDA tensors"),
+    ]
+    for fn, msg in cases:
+        with pytest.raises(ValueError, match=msg):
+            fn()

@@ -3,8 +3,10 @@
 Callers that cannot allocate device memory (a runtime with a fixed arena, a loop
 that must not touch the allocator) use this variant; its scratch is a fixed
 array inside the library.  It must give the same factor and order as
-gptq_factor_hessian, on repeated calls (the shared scratch keeps the previous
-call's contents), and reject sizes above its capacity.
+gptq_factor_hessian, bit for bit (both run the same deterministic kernels), on
+repeated calls (the shared scratch keeps the previous call's contents); once
+the library's code is loaded on the device, a call must not change the device's
+free memory; and sizes above its capacity are rejected.
 
 This file is collected last on purpose, so a run that stops at the first
 failure has already run every other test.
@@ -66,7 +68,25 @@ def test_matches_pooled_entry_point_on_two_calls(n, desc_act):
         a, b = U.cpu().numpy(), U_ref.cpu().numpy()
         err = np.abs(a - b).max(axis=1) / np.abs(b).max(axis=1)
         assert err.max() <= U_RTOL
+        assert torch.equal(U, U_ref)  # same kernels, deterministic: identical bits
         assert np.all(np.tril(a, -1) == 0)
+
+
+def test_a_call_allocates_no_device_memory():
+    """After a first call (which may load the library's code, and with it the fixed array,
+    onto the device), further calls leave the device's free memory unchanged."""
+    dev = torch.device("cuda:0")
+    L, f = _fn()
+    n = 512
+    Hd = _hessian(n, 2 * n, 77).to(dev)
+    U = torch.empty(n, n, dtype=torch.float64, device=dev)
+    perm = torch.empty(n, dtype=torch.int32, device=dev)
+    assert _call(f, Hd, 0.01, 1, U, perm) == 0  # warm-up: module load
+    free0, _ = torch.cuda.mem_get_info(dev)
+    for desc_act in (1, 0):
+        assert _call(f, Hd, 0.01, desc_act, U, perm) == 0
+    free1, _ = torch.cuda.mem_get_info(dev)
+    assert free1 == free0, (free0, free1)
 
 
 def test_rejects_sizes_beyond_capacity():
