@@ -35,6 +35,7 @@ Readings taken where the pages are silent:
 from __future__ import annotations
 
 import numpy as np
+from scipy.linalg import lapack as _lapack
 
 __all__ = [
     "NotPositiveDefinite",
@@ -151,18 +152,21 @@ def inverse_cholesky_upper(Hd):
     Hd = np.asarray(Hd, dtype=np.float64)
     if not np.all(np.isfinite(Hd)):
         raise NotPositiveDefinite("non-finite entries in the damped Hessian")
-    try:
-        np.linalg.cholesky(Hd)
-    except np.linalg.LinAlgError as exc:
-        raise NotPositiveDefinite(str(exc)) from exc
-    n = Hd.shape[0]
-    Hinv = np.linalg.solve(Hd, np.eye(n))
-    Hinv = 0.5 * (Hinv + Hinv.T)
-    try:
-        L = np.linalg.cholesky(Hinv)  # Hinv = L L^T
-    except np.linalg.LinAlgError as exc:
-        raise NotPositiveDefinite(str(exc)) from exc
-    return L.T.copy()  # U = L^T, Hinv = U^T U
+    # inverse(Hd) of a symmetric positive definite matrix, formed from its own Cholesky
+    # factor (LAPACK potrf, then potri, upper triangles); potrf's failure is the
+    # not-positive-definite case
+    C, info = _lapack.dpotrf(Hd, lower=0, clean=1)
+    if info != 0:
+        raise NotPositiveDefinite(f"Cholesky of the damped Hessian failed (potrf info {info})")
+    Hinv, info = _lapack.dpotri(C, lower=0)  # upper triangle of inverse(Hd)
+    if info != 0:
+        raise NotPositiveDefinite(f"inverse of the damped Hessian failed (potri info {info})")
+    # Cholesky factor of the inverse: upper U with inverse(Hd) = U^T U (potrf reads the
+    # upper triangle only)
+    U, info = _lapack.dpotrf(Hinv, lower=0, clean=1)
+    if info != 0:
+        raise NotPositiveDefinite(f"Cholesky of the inverse failed (potrf info {info})")
+    return U
 
 
 # --------------------------------------------------------------------------- quantizer
