@@ -54,6 +54,10 @@ __all__ = [
     "pack",
     "unpack",
     "dequantize",
+    "export_tensors",
+    "dequantize_checkpoint",
+    "round16",
+    "quantized_linear",
     "layer_loss",
     "layer_loss_h",
     "brute_force_min_loss",
@@ -166,7 +170,7 @@ def inverse_cholesky_upper(Hd):
     U, info = _lapack.dpotrf(Hinv, lower=0, clean=1)
     if info != 0:
         raise NotPositiveDefinite(f"Cholesky of the inverse failed (potrf info {info})")
-    return U
+    return np.ascontiguousarray(U)  # LAPACK returns column-major storage
 
 
 # --------------------------------------------------------------------------- quantizer
@@ -434,6 +438,51 @@ def unpack(qweight, bits, n_in):
             v |= q[w + 1] << np.uint64(32 - off)
         codes[:, c] = (v & mask).astype(np.int64)
     return codes
+
+
+def export_tensors(scales, zeros, bits):
+    """Checkpoint form of a linear's group parameters: (fp16 scales, packed zero points).
+
+    [examples §1.4; OLMo §四 step 4]: save_quantized stores the quantized weights with
+    their scale and zero point; the pages give no tensor layout.  Layout of this library:
+    scales rounded to IEEE half precision (round to nearest even), and for each group
+    the zero points of the output channels packed as :func:`pack` packs codes, along
+    n_out: qzeros [G, n_out*bits/32].
+    """
+    S = np.asarray(scales, dtype=np.float32).astype(np.float16)
+    Z = np.asarray(zeros, dtype=np.int64)
+    return S, pack(Z, bits).T.copy()
+
+
+def dequantize_checkpoint(qweight, qzeros, scales16, g_idx, bits):
+    """Exact dequantized weight [n_out, n_in] of the checkpoint form (float64).
+
+    [ch5 §5.1.1]: x_hat = s * (q - z), per weight with its group's half-precision scale
+    and packed zero point (the layout of :func:`export_tensors`):
+    W_hat[o, c] = scales16[g_idx[c], o] * (code[o, c] - zero[g_idx[c], o]).
+    """
+    g = np.asarray(g_idx, dtype=np.int64)
+    n_in = g.shape[0]
+    S = np.asarray(scales16, dtype=np.float16).astype(np.float64)
+    n_out = S.shape[1]
+    Z = unpack(np.asarray(qzeros).T, bits, n_out)  # [G, n_out]
+    codes = unpack(qweight, bits, n_in)
+    return S[g, :].T * (codes - Z[g, :].T)
+
+
+def round16(A, dtype):
+    """Round to the nearest 16-bit value ("float16" or "bfloat16"), ties to even; returned
+    as float64.  The operand precision of a 16-bit tensor-core multiply."""
+    A = np.asarray(A, dtype=np.float64)
+    if dtype == "float16":
+        return A.astype(np.float16).astype(np.float64)
+    import torch  # the bfloat16 conversion of plain PyTorch on the CPU
+    return torch.from_numpy(A).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+def quantized_linear(X, What16):
+    """Y = X W^T in float64 (X [M, n_in] 16-bit values, What16 the rounded weight)."""
+    return np.asarray(X, np.float64) @ np.asarray(What16, np.float64).T
 
 
 def dequantize(qweight, scales, zeros, g_idx, bits, n_in):

@@ -30,7 +30,8 @@ class LayerTimes:
         return self.hessian_ms + self.factor_ms + self.sweep_ms
 
 
-def quantize_decoder_layer(acts, weights, modules, qcfg, hessians=None, timing=False, stream=None):
+def quantize_decoder_layer(acts, weights, modules, qcfg, hessians=None, timing=False, stream=None,
+                           hessians_given=False):
     """Quantize the linears of one decoder layer.
 
     acts:     {h_index: X [tokens, n] fp16/bf16 CUDA tensor, or a list of token chunks}
@@ -38,6 +39,9 @@ def quantize_decoder_layer(acts, weights, modules, qcfg, hessians=None, timing=F
     modules:  iterable of objects with .name and .h_index
     qcfg:     object with bits, group_size, damp_percent, sym, desc_act, static_groups, blocksize
     hessians: optional {h_index: preallocated [n, n] fp32 CUDA tensor} (zeroed here)
+    hessians_given: the `hessians` already hold the layer's Hessians (accumulated earlier,
+              e.g. streamed chunk by chunk); `acts` is then ignored and nothing is
+              accumulated.
     Returns ({module name: QuantResult}, LayerTimes or None).
     """
     stream = stream or torch.cuda.current_stream()
@@ -57,7 +61,11 @@ def quantize_decoder_layer(acts, weights, modules, qcfg, hessians=None, timing=F
         mark()
         Hs = {}
         launch_marks = []
-        for h, X in acts.items():
+        if hessians_given:
+            if not hessians:
+                raise ValueError("hessians_given needs the layer's Hessians in `hessians`")
+            Hs = dict(hessians)
+        for h, X in ({} if hessians_given else acts).items():
             chunks = X if isinstance(X, (list, tuple)) else [X]
             n = chunks[0].shape[1]
             H = hessians[h] if hessians is not None else torch.empty(n, n, dtype=torch.float32, device=chunks[0].device)

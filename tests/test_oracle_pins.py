@@ -364,3 +364,85 @@ def test_tiny_config_end_to_end_runs():
     assert out["scales"].shape == (8, 64)
     assert O.layer_loss(W, out["What"], X) < O.layer_loss(W, What_rtn, X)
     assert torch.float16 == cfg.x_dtype
+
+
+def test_sweep_identity_check_is_complete_and_catches_planted_mistakes():
+    """The per-decision sweep check used at order 28672 (tests/sweep_identities.py):
+    the oracle's own outputs pass every decision, and a sweep run with a mistake planted in
+    the oracle (two rows of U scaled, or all compensation dropped) fails it."""
+    import torch
+
+    from post_weight_quantization_layer_b200 import synth
+    from tests.sweep_identities import sweep_decisions
+    n_out, n, g, bits, sym = 6, 512, 128, 4, True
+    W = synth.outlier_weight(n_out, n, 5).double().numpy()
+    X = synth.StudentTActs(n, 4 * n, 9, dtype=torch.bfloat16).full().double().numpy()
+    H = O.hessian(X).astype(np.float32).astype(np.float64)
+    out = O.gptq_quantize(W, H, bits, g, 0.01, sym, False, False, 128)
+    U = out["U"]
+    p_ok, c_ok = sweep_decisions(W, out["What"], out["codes"], out["scales"], out["zeros"], U, bits, sym, g)
+    assert p_ok == 1.0 and c_ok == 1.0
+    for planted in ("scaled_rows", "no_compensation"):
+        Ub = U.copy()
+        if planted == "scaled_rows":
+            Ub[100, 101:] *= 1.3
+            Ub[300, 301:] *= 1.3
+        else:
+            Ub = np.diag(np.diag(U))
+        bad = O.gptq_sweep(W, Ub, bits, sym, g, np.arange(n), False, W, 128)
+        assert np.mean(bad["codes"] == out["codes"]) < 1.0
+        p_b, c_b = sweep_decisions(W, bad["xhat"], bad["codes"], bad["scales"], bad["zeros"], U, bits, sym, g)
+        assert c_b < 0.9999, (planted, c_b)
+
+
+def test_export_tensors_hand_words():
+    """Packed zero points and fp16 scales of the checkpoint form against hand-built words
+    (tests/golden/export.txt)."""
+    cases = {"seq4": (4, np.array([np.arange(1, 9), np.full(8, 8)])),
+             "cyc2": (2, (np.arange(16) % 4)[None, :]),
+             "byte8": (8, np.array([[1, 2, 3, 4]]))}
+    for ln in read_golden("export.txt"):
+        f = ln.split()
+        if f[0] == "bf16":
+            continue
+        if f[0] == "half":
+            S, _ = O.export_tensors(np.full((1, 8), float(f[1])), np.zeros((1, 8), np.int64), 4)
+            assert S.dtype == np.float16
+            assert np.all(S.view(np.uint16) == int(f[2], 16)), ln
+            continue
+        bits, zeros = cases[f[0]]
+        _, qz = O.export_tensors(np.ones(zeros.shape), zeros, bits)
+        assert qz.shape == (zeros.shape[0], zeros.shape[1] * bits // 32)
+        assert qz.view(np.uint32)[int(f[2]), int(f[3])] == int(f[4], 16), ln
+
+
+def test_round16_hand_cases():
+    """bfloat16 / float16 rounding of the oracle against hand-derived ties
+    (tests/golden/export.txt)."""
+    for ln in read_golden("export.txt"):
+        f = ln.split()
+        if f[0] == "bf16":
+            assert O.round16(np.array([float(f[1])]), "bfloat16")[0] == float(f[2]), ln
+        elif f[0] == "half":
+            v = O.round16(np.array([float(f[1])]), "float16")[0]
+            assert np.float16(v).view(np.uint16) == int(f[2], 16), ln
+
+
+def test_dequantize_checkpoint_matches_codes_and_params():
+    """The checkpoint form dequantizes to s16[g] * (q - z[g]) element by element, for any
+    g_idx order (act order), against a loop over single weights."""
+    rng = np.random.default_rng(12)
+    for bits in (2, 4, 8):
+        n_out, n_in, G = 16, 64, 4
+        codes = rng.integers(0, 2**bits, size=(n_out, n_in))
+        zeros = rng.integers(0, 2**bits, size=(G, n_out))
+        scales = rng.random((G, n_out)) * 0.1
+        g_idx = rng.permutation(np.arange(n_in) // (n_in // G))
+        S16, qz = O.export_tensors(scales, zeros, bits)
+        W = O.dequantize_checkpoint(O.pack(codes, bits), qz, S16, g_idx, bits)
+        for o in range(0, n_out, 5):
+            for c in range(0, n_in, 7):
+                g = g_idx[c]
+                assert W[o, c] == float(S16[g, o]) * (codes[o, c] - zeros[g, o])
+        Y = O.quantized_linear(np.eye(n_in)[:3], W)
+        assert np.array_equal(Y, W[:, :3].T)
