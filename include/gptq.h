@@ -187,6 +187,93 @@ int gptq_quantize_layer_factored(const void* W, int w_dtype, int64_t n_out, int6
                                  int32_t* g_idx, void* stream, gptq_stats* stats);
 
 /*
+ * Checkpoint form of one quantized linear: half-precision scales and packed zero points.
+ * Source: AutoGPTQ examples guide §1.4 and the OLMo quick-start §四 step 4
+ * (save_quantized stores the quantized weights, with scale and zero point, beside
+ * quantize_config.json); the pages give no tensor layout, so the layout is this library's.
+ *
+ * scales     [groups, n_out] fp32 (as written by gptq_quantize_layer), read-only.
+ * zeros      [groups, n_out] int32 zero points in [0, 2^bits - 1], read-only (only the low
+ *            `bits` bits of each value are stored).
+ * scales_f16 [groups, n_out] fp16 output (IEEE binary16 bits), round to nearest even.
+ * qzeros     [groups, n_out*bits/32] int32 output: for each group, the zero points of the
+ *            output channels form an LSB-first stream of bits-wide fields cut into 32-bit
+ *            words (the packing of qweight, along n_out; 3-bit fields straddle words).
+ * qweight and g_idx are stored as gptq_quantize_layer wrote them.
+ * bits not in {2,3,4,8}, groups or n_out <= 0, NULL pointers -> INVALID_ARG;
+ * n_out*bits % 32 != 0, groups > 65535 or pointers not 16-byte aligned -> UNSUPPORTED.
+ * Asynchronous on `stream`.
+ */
+int gptq_export_layer(const float* scales, const int32_t* zeros, int64_t groups, int64_t n_out, int bits,
+                      uint16_t* scales_f16, int32_t* qzeros, void* stream);
+
+/*
+ * Dequantize a checkpoint-form linear into a dense 16-bit weight W [n_out, n_in]
+ * (a torch.nn.Linear weight): W[n, k] = round16(scales[g_idx[k], n] * (code[k, n] -
+ * zero[g_idx[k], n])), rounded once to nearest even in out_dtype (GPTQ_F16 or GPTQ_BF16).
+ * Source: the dequantized weight of chapter 5 §5.1.1 (x_hat = s * (q - z)) applied to the
+ * checkpoint tensors of gptq_export_layer.
+ *
+ * qweight [n_in*bits/32, n_out] int32, qzeros [groups, n_out*bits/32] int32, scales_f16
+ * [groups, n_out] fp16, g_idx [n_in] int32 (any order; entries outside [0, groups) are
+ * clamped into it), all read-only.  bits 2, 4 or 8 (3 -> UNSUPPORTED: its fields straddle
+ * words).  n_in % 64 == 0, n_out % 8 == 0 and n_out * bits % 32 == 0 (whole words of zero
+ * points), else UNSUPPORTED.  Asynchronous on `stream`.
+ */
+int gptq_dequantize_weight(const int32_t* qweight, const int32_t* qzeros, const uint16_t* scales_f16,
+                           const int32_t* g_idx, int64_t groups, int64_t n_in, int64_t n_out, int bits,
+                           int out_dtype, void* W, void* stream);
+
+/*
+ * Linear layer on quantized weights (weight-only quantization, 16-bit activations):
+ * Y = X * round16(W_hat)^T, W_hat as in gptq_dequantize_weight, products accumulated in
+ * fp32, Y rounded to x_dtype.  The inference side of the quantized checkpoint ("gptq"
+ * skill card, kernel backends; chapter 5 §5.2 generation speed).
+ *
+ * X [M, n_in] fp16 or bf16 (x_dtype), Y [M, n_out] of the same dtype; M >= 0 (0: no-op,
+ * X and Y may then be NULL).
+ * Weight arguments as in gptq_dequantize_weight.
+ * M <= 4 (decoding): one pass over the packed weights, dequantized in registers, K split
+ * over CTAs and the splits added in a fixed order (deterministic).  M > 4: the weights are
+ * dequantized once into a 16-bit workspace (library pool, n_in*n_out*2 bytes) and
+ * multiplied on the tensor cores (tcgen05, fp32 accumulate in TMEM); deterministic.
+ * Asynchronous on `stream`; a bounded device wait that gives up is reported by
+ * gptq_device_status.
+ */
+int gptq_quantized_linear(const void* X, int x_dtype, int64_t M, int64_t n_in, const int32_t* qweight,
+                          const int32_t* qzeros, const uint16_t* scales_f16, const int32_t* g_idx,
+                          int64_t groups, int64_t n_out, int bits, void* Y, void* stream);
+
+/*
+ * Forward pieces of a Llama-style decoder layer, used to quantize its linears in execution
+ * order (true_sequential: AutoGPTQ examples guide §1.4, OLMo quick-start §三): the
+ * calibration input of each linear is produced by the layer's earlier modules with their
+ * weights already quantized.  The pages do not spell the block out; the Llama-2 block is
+ *   x = rmsnorm(h); h1 = h + o_proj(attention(rope(q_proj x), rope(k_proj x), v_proj x));
+ *   y = rmsnorm(h1); h2 = h1 + down_proj(silu(gate_proj y) * up_proj y).
+ * All tensors are 16-bit (dtype GPTQ_F16 or GPTQ_BF16), row-major, one row per token;
+ * arithmetic is fp32 and every output is rounded to nearest even.  Asynchronous on
+ * `stream`.  Bad sizes, dtypes or NULL pointers -> INVALID_ARG.
+ */
+/* y[r, :] = x[r, :] / sqrt(mean(x[r, :]^2) + eps) * gamma, x and y [rows, dim], gamma [dim]. */
+int gptq_rmsnorm(const void* x, int dtype, int64_t rows, int64_t dim, const void* gamma, float eps, void* y,
+                 void* stream);
+/* Rotary position embedding, in place on x [tokens, heads * head_dim]: in each head the
+ * pairs (i, i + head_dim/2) rotate by pos * base^(-2i/head_dim), pos = token index modulo
+ * seq_len (tokens are whole sequences of seq_len); angles in double precision. */
+int gptq_rope(void* x, int dtype, int64_t tokens, int heads, int head_dim, int seq_len, double base,
+              void* stream);
+/* Causal attention per sequence and head: out = softmax(q k^T / sqrt(head_dim), keys at or
+ * before the query) v; q, k, v, out [tokens, heads * head_dim], tokens a multiple of
+ * seq_len; head_dim % 4 == 0 and <= 128 (else UNSUPPORTED above 128). */
+int gptq_attention(const void* q, const void* k, const void* v, int dtype, int64_t tokens, int heads,
+                   int head_dim, int seq_len, void* out, void* stream);
+/* out = gate / (1 + exp(-gate)) * up, elementwise over `count` values. */
+int gptq_silu_mul(const void* gate, const void* up, int dtype, int64_t count, void* out, void* stream);
+/* out = a + b, elementwise over `count` values (the residual connection). */
+int gptq_add(const void* a, const void* b, int dtype, int64_t count, void* out, void* stream);
+
+/*
  * gptq_factor_hessian for callers that cannot allocate device memory.
  * The paper has no counterpart: this is a deployment variant of the factor call.
  *
@@ -232,6 +319,18 @@ int gptq_trim_workspace(void);
  * clear != 0 resets it to GPTQ_OK afterwards.
  */
 int gptq_device_status(void* stream, int clear);
+
+/*
+ * Test switch for the expiry path of the bounded device-side waits (off by default; no
+ * counterpart on the pages).  With skip_loads != 0, later gptq_accumulate_hessian launches
+ * issue no loads of X, so the kernel's waits for data run out after wait_limit polls each:
+ * the kernel records GPTQ_ERR_TIMEOUT (read by gptq_device_status), releases its tensor
+ * memory and returns normally, leaving H unchanged and the context usable.  wait_limit != 0
+ * also replaces the default limit (2^24 polls) for normal launches; (0, 0) restores the
+ * defaults.  skip_loads != 0 with wait_limit == 0 -> INVALID_ARG (the expiry test always
+ * uses a short limit).  Process-wide; meant for tests.
+ */
+int gptq_test_wait_expiry(int skip_loads, uint32_t wait_limit);
 
 /* Static description of a status code (never NULL). */
 const char* gptq_status_string(int status);

@@ -11,6 +11,7 @@ from .api import (  # noqa: F401
     GPTQError,
     QuantResult,
     accumulate_hessian,
+    dequantize_weight,
     device_status,
     factor_hessian,
     factor_hessians,
@@ -18,6 +19,7 @@ from .api import (  # noqa: F401
     launch_count,
     quantize_layer,
     quantize_layer_factored,
+    quantized_linear,
 )
 
 __version__ = "0.1.0"

@@ -48,6 +48,17 @@ _SIGNATURES = {
     "gptq_quantize_layer_factored": (c_int, [c_void_p, c_int, c_i64, c_i64, c_void_p, c_void_p, c_int, c_int,
                                              c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
                                              c_void_p, ctypes.POINTER(GptqStats)]),
+    "gptq_export_layer": (c_int, [c_void_p, c_void_p, c_i64, c_i64, c_int, c_void_p, c_void_p, c_void_p]),
+    "gptq_dequantize_weight": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_i64, c_i64, c_i64, c_int, c_int,
+                                       c_void_p, c_void_p]),
+    "gptq_quantized_linear": (c_int, [c_void_p, c_int, c_i64, c_i64, c_void_p, c_void_p, c_void_p, c_void_p, c_i64,
+                                      c_i64, c_int, c_void_p, c_void_p]),
+    "gptq_test_wait_expiry": (c_int, [c_int, ctypes.c_uint32]),
+    "gptq_rmsnorm": (c_int, [c_void_p, c_int, c_i64, c_i64, c_void_p, c_float, c_void_p, c_void_p]),
+    "gptq_rope": (c_int, [c_void_p, c_int, c_i64, c_int, c_int, c_int, ctypes.c_double, c_void_p]),
+    "gptq_attention": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_i64, c_int, c_int, c_int, c_void_p, c_void_p]),
+    "gptq_silu_mul": (c_int, [c_void_p, c_void_p, c_int, c_i64, c_void_p, c_void_p]),
+    "gptq_add": (c_int, [c_void_p, c_void_p, c_int, c_i64, c_void_p, c_void_p]),
     "gptq_device_status": (c_int, [c_void_p, c_int]),
     "gptq_trim_workspace": (c_int, []),
     "gptq_status_string": (ctypes.c_char_p, [c_int]),

@@ -204,3 +204,120 @@ def quantize_layer_factored(W, U, perm, bits=4, group_size=128, sym=True, static
         ctypes.byref(st_obj) if stats else None)
     _check(st, "gptq_quantize_layer_factored")
     return QuantResult(qw, sc, zr, gi, _stats_dict(st_obj) if stats else None)
+
+
+def _checkpoint(ck, bits):
+    """(qweight, qzeros, scales, g_idx, groups, n_in, n_out) of a checkpoint-form linear
+    (the dict of export.export_layer / export.load_quantized), checked."""
+    try:
+        qw, qz, sc, gi = ck["qweight"], ck["qzeros"], ck["scales"], ck["g_idx"]
+    except (KeyError, TypeError):
+        raise ValueError("checkpoint linear needs qweight, qzeros, scales and g_idx") from None
+    if not isinstance(gi, torch.Tensor) or gi.dim() != 1:
+        raise ValueError("g_idx must be a 1-D int32 tensor")
+    n_in = gi.shape[0]
+    if not isinstance(sc, torch.Tensor) or sc.dim() != 2:
+        raise ValueError("scales must be a 2-D [groups, n_out] float16 tensor")
+    G, n_out = sc.shape
+    _need(qw, "qweight", (torch.int32,), (n_in * bits // 32, n_out))
+    _need(qz, "qzeros", (torch.int32,), (G, n_out * bits // 32))
+    _need(sc, "scales", (torch.float16,), (G, n_out))
+    _need(gi, "g_idx", (torch.int32,), (n_in,))
+    return qw, qz, sc, gi, G, n_in, n_out
+
+
+def dequantize_weight(ck, bits=4, dtype=torch.float16, stream=None):
+    """Dense [n_out, n_in] weight of a checkpoint-form linear, each value rounded once to
+    `dtype` (float16 or bfloat16)."""
+    qw, qz, sc, gi, G, n_in, n_out = _checkpoint(ck, bits)
+    if dtype not in (torch.float16, torch.bfloat16):
+        raise ValueError("dtype must be float16 or bfloat16")
+    _need_cuda(qw, qz, sc, gi)
+    W = torch.empty(n_out, n_in, dtype=dtype, device=qw.device)
+    st = lib().gptq_dequantize_weight(_ptr(qw), _ptr(qz), _ptr(sc), _ptr(gi), G, n_in, n_out, bits, _DTYPE[dtype],
+                                      _ptr(W), _stream(stream))
+    _check(st, "gptq_dequantize_weight")
+    return W
+
+
+def quantized_linear(X, ck, bits=4, out=None, stream=None):
+    """Y = X W_hat^T for X [M, n_in] (float16 or bfloat16) and a checkpoint-form linear."""
+    qw, qz, sc, gi, G, n_in, n_out = _checkpoint(ck, bits)
+    if not isinstance(X, torch.Tensor) or X.dim() != 2:
+        raise ValueError("X must be a 2-D [M, n_in] tensor")
+    _need(X, "X", (torch.float16, torch.bfloat16), (X.shape[0], n_in))
+    M = X.shape[0]
+    if out is None:
+        out = torch.empty(M, n_out, dtype=X.dtype, device=X.device)
+    _need(out, "out", (X.dtype,), (M, n_out))
+    _need_cuda(X, out, qw, qz, sc, gi)
+    st = lib().gptq_quantized_linear(_ptr(X), _DTYPE[X.dtype], M, n_in, _ptr(qw), _ptr(qz), _ptr(sc), _ptr(gi), G,
+                                     n_out, bits, _ptr(out), _stream(stream))
+    _check(st, "gptq_quantized_linear")
+    return out
+
+
+# ------------------------------------------------------------------ decoder-layer forward pieces
+def _act(x, what):
+    if not isinstance(x, torch.Tensor) or x.dtype not in (torch.float16, torch.bfloat16):
+        raise ValueError(f"{what} must be a float16 or bfloat16 tensor")
+    return x
+
+
+def rmsnorm(x, gamma, eps=1e-5, stream=None):
+    """x / sqrt(mean(x^2) + eps) * gamma over the last dimension of x [rows, dim]."""
+    _act(x, "x")
+    if x.dim() != 2:
+        raise ValueError("x must be [rows, dim]")
+    _need(gamma, "gamma", (x.dtype,), (x.shape[1],))
+    y = torch.empty_like(x)
+    _need_cuda(x, gamma, y)
+    _check(lib().gptq_rmsnorm(_ptr(x), _DTYPE[x.dtype], x.shape[0], x.shape[1], _ptr(gamma), float(eps), _ptr(y),
+                              _stream(stream)), "gptq_rmsnorm")
+    return y
+
+
+def rope_(x, heads, seq_len, base=10000.0, stream=None):
+    """Rotary embedding in place on x [tokens, heads * head_dim] (tokens = whole sequences)."""
+    _act(x, "x")
+    if x.dim() != 2 or x.shape[1] % heads:
+        raise ValueError("x must be [tokens, heads * head_dim]")
+    _need_cuda(x)
+    _check(lib().gptq_rope(_ptr(x), _DTYPE[x.dtype], x.shape[0], heads, x.shape[1] // heads, seq_len, float(base),
+                           _stream(stream)), "gptq_rope")
+    return x
+
+
+def attention(q, k, v, heads, seq_len, stream=None):
+    """Causal softmax attention per sequence and head; q, k, v [tokens, heads * head_dim]."""
+    _act(q, "q")
+    if q.dim() != 2 or q.shape[1] % heads:
+        raise ValueError("q must be [tokens, heads * head_dim]")
+    _need(k, "k", (q.dtype,), tuple(q.shape))
+    _need(v, "v", (q.dtype,), tuple(q.shape))
+    out = torch.empty_like(q)
+    _need_cuda(q, k, v, out)
+    _check(lib().gptq_attention(_ptr(q), _ptr(k), _ptr(v), _DTYPE[q.dtype], q.shape[0], heads, q.shape[1] // heads,
+                                seq_len, _ptr(out), _stream(stream)), "gptq_attention")
+    return out
+
+
+def silu_mul(gate, up, stream=None):
+    """gate / (1 + exp(-gate)) * up, elementwise."""
+    _act(gate, "gate")
+    _need(up, "up", (gate.dtype,), tuple(gate.shape))
+    out = torch.empty_like(gate)
+    _need_cuda(gate, up, out)
+    _check(lib().gptq_silu_mul(_ptr(gate), _ptr(up), _DTYPE[gate.dtype], gate.numel(), _ptr(out), _stream(stream)),
+           "gptq_silu_mul")
+    return out
+
+
+def add(a, b, stream=None):
+    """a + b, elementwise (the residual connection)."""
+    _act(a, "a")
+    _need(b, "b", (a.dtype,), tuple(a.shape))
+    out = torch.empty_like(a)
+    _need_cuda(a, b, out)
+    _check(lib().gptq_add(_ptr(a), _ptr(b), _DTYPE[a.dtype], a.numel(), _ptr(out), _stream(stream)), "gptq_add")
+    return out

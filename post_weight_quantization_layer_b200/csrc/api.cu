@@ -209,6 +209,23 @@ int factor_on_lanes(const float* H, int64_t n, float damp, bool desc_act, double
 }
 
 }  // namespace
+
+int pool_alloc(void** p, size_t bytes, cudaStream_t s) {
+  *p = nullptr;
+  cudaMemPool_t pool = workspace_pool();
+  if (!pool) return GPTQ_ERR_CUDA;
+  if (cudaMallocFromPoolAsync(p, bytes, pool, s) != cudaSuccess) {
+    cudaGetLastError();
+    *p = nullptr;
+    return GPTQ_ERR_OOM;
+  }
+  return GPTQ_OK;
+}
+
+void pool_free(void* p, cudaStream_t s) {
+  if (p) cudaFreeAsync(p, s);
+}
+
 }  // namespace gptq
 
 using namespace gptq;
@@ -250,8 +267,16 @@ int gptq_trim_workspace(void) {
   return cudaMemPoolTrimTo(pool, 0) == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
 }
 
+int gptq_test_wait_expiry(int skip_loads, uint32_t wait_limit) {
+  if (skip_loads && wait_limit == 0) return GPTQ_ERR_INVALID_ARG;  // only with a short limit
+  hessian_wait_test(skip_loads, wait_limit);
+  return GPTQ_OK;
+}
+
 int gptq_device_status(void* stream, int clear) {
-  return hessian_device_status(static_cast<cudaStream_t>(stream), clear);
+  const int h = hessian_device_status(static_cast<cudaStream_t>(stream), clear);
+  const int g = gemm_device_status(clear);
+  return h != GPTQ_OK ? h : g;
 }
 
 int gptq_factor_hessian(const float* H, int64_t n_in, float damp_percent, int desc_act, double* U, int32_t* perm,

@@ -37,9 +37,11 @@ inline int after_launch() {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Raise a kernel's dynamic shared-memory limit to `bytes` on the current device.  The
-// attribute is per device, so it is set once for every (device, kernel) pair this process
-// launches on; a process may drive several GPUs.  Thread-safe.
+// Make a kernel's dynamic shared-memory limit on the current device at least `bytes`.  The
+// attribute is per device: it is raised for every (device, kernel) pair this process
+// launches on (a process may drive several GPUs) whenever a launch needs more than the
+// limit set so far (kernels whose shared memory depends on the call's sizes).
+// Thread-safe.
 int ensure_smem_limit(const void* kernel, int bytes);
 
 inline int num_sms() {
@@ -68,6 +70,13 @@ constexpr int kStatusTimeout = GPTQ_ERR_TIMEOUT;
 // hessian.cu
 int launch_hessian(const void* X, int x_dtype, int64_t tokens, int64_t n, float* H, cudaStream_t s);
 int hessian_device_status(cudaStream_t s, int clear);
+void hessian_wait_test(int skip_loads, uint32_t wait_limit);
+
+// w4a16.cu: Y[M, N] = X[M, K] * Wd[N, K]^T, 16-bit operands (x_dtype), fp32 accumulate, on the
+// tcgen05 tensor cores; and its bounded-wait status word.
+int gemm_bf16_tn(const void* X, const void* Wd, void* Y, int64_t M, int64_t N, int64_t K, int x_dtype,
+                 cudaStream_t s);
+int gemm_device_status(int clear);
 
 // gemm.cu: fp64 C[m,n] = beta*C[m,n] + alpha * sum_k A[m*lda+k] * B(k,n),
 // B(k,n) = transB ? B[n*ldb+k] : B[k*ldb+n].  upper != 0 skips tiles of C lying entirely
@@ -116,6 +125,11 @@ struct SweepArgs {
   cudaEvent_t ev[4];      // valid when stats != null
 };
 int run_sweep(SweepArgs& a, cudaStream_t s, int* panel_width, int* outer_width);
+
+// api.cu: stream-ordered allocation from the library's workspace pool (one pool per device,
+// memory kept cached between calls).  pool_alloc returns GPTQ_ERR_OOM on failure.
+int pool_alloc(void** p, size_t bytes, cudaStream_t s);
+void pool_free(void* p, cudaStream_t s);
 
 // lanes.cu: library-owned streams leased by one call (see the file's header).
 enum LanePrio { kLaneHigh = 0, kLaneLow = 1 };

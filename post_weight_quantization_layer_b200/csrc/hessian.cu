@@ -24,6 +24,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -46,14 +47,25 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;     // 48 KiB
 constexpr int FLUSH_KSTEPS = 16;                   // drain every 1024 tokens
 constexpr int THREADS = 320;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
-constexpr uint32_t WAIT_LIMIT = 1u << 24;
+constexpr uint32_t kWaitLimit = 1u << 24;  // polls before a wait gives up (normal runs)
 
 __device__ int g_hessian_status = 0;
+
+// Expiry test of the bounded waits (host-set, off by default): the producer issues no load,
+// so the MMA and drain warps' waits run out after `wait_limit` polls; the CTA then records
+// GPTQ_ERR_TIMEOUT, frees its TMEM and returns, and H is left unchanged.
+struct WaitTest {
+  int skip_loads;
+  uint32_t wait_limit;
+};
+std::atomic<int> g_test_skip{0};
+std::atomic<uint32_t> g_test_limit{0};
 
 template <uint32_t AB_FMT>
 __global__ void __launch_bounds__(THREADS, 1)
     hessian_syrk_kernel(const __grid_constant__ CUtensorMap tmap, float* __restrict__ H, int n, int64_t T,
-                        int tiles, int S, int64_t tok_per_seg) {
+                        int tiles, int S, int64_t tok_per_seg, WaitTest wt) {
+  const uint32_t WAIT_LIMIT = wt.wait_limit;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
@@ -104,7 +116,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       int stage = 0;
       uint32_t ph = 0;
       int issued = 0;
-      for (int u = blockIdx.x; u < units && ok; u += G) {
+      for (int u = blockIdx.x; u < units && ok && !wt.skip_loads; u += G) {
         int tile;
         int64_t t0;
         const int nk = unit_ksteps(u, tile, t0);
@@ -185,6 +197,9 @@ __global__ void __launch_bounds__(THREADS, 1)
               ph ^= 1u;
             }
           }
+          // after a failed wait the accumulator is incomplete: never hand it to the drain
+          // warps (their own bounded wait then runs out and nothing is added to H)
+          if (!ok) break;
           umma_commit(&accf[b]);
         }
       }
@@ -340,7 +355,9 @@ int launch_impl(const void* X, int64_t T, int n, float* H, cudaStream_t st) {
     const int S = static_cast<int>((Tc + tok_per_seg - 1) / tok_per_seg);  // no empty segments
     if (static_cast<int64_t>(tiles) * S >= (int64_t(1) << 31)) return GPTQ_ERR_UNSUPPORTED;
     const int G = static_cast<int>(std::min<int64_t>(sms, static_cast<int64_t>(tiles) * S));
-    hessian_syrk_kernel<F><<<G, THREADS, SMEM_BYTES, st>>>(tm, H, n, Tc, tiles, S, tok_per_seg);
+    const uint32_t lim = g_test_limit.load();
+    const WaitTest wt{g_test_skip.load(), lim ? lim : kWaitLimit};
+    hessian_syrk_kernel<F><<<G, THREADS, SMEM_BYTES, st>>>(tm, H, n, Tc, tiles, S, tok_per_seg, wt);
     GPTQ_TRY(after_launch());
   }
   return GPTQ_OK;
@@ -351,6 +368,11 @@ int launch_impl(const void* X, int64_t T, int n, float* H, cudaStream_t st) {
 int launch_hessian(const void* X, int x_dtype, int64_t tokens, int64_t n, float* H, cudaStream_t s) {
   if (x_dtype == GPTQ_BF16) return launch_impl<1>(X, tokens, static_cast<int>(n), H, s);
   return launch_impl<0>(X, tokens, static_cast<int>(n), H, s);
+}
+
+void hessian_wait_test(int skip_loads, uint32_t wait_limit) {
+  g_test_skip.store(skip_loads ? 1 : 0);
+  g_test_limit.store(wait_limit);
 }
 
 int hessian_device_status(cudaStream_t s, int clear) {

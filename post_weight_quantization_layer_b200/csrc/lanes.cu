@@ -10,7 +10,6 @@
 // workspace on the caller's stream never overtake a lane.
 #include <map>
 #include <mutex>
-#include <set>
 #include <vector>
 
 #include "common.cuh"
@@ -74,19 +73,20 @@ int LaneLease::acquire(int count, const LanePrio* prio) {
 
 namespace {
 std::mutex g_attr_mu;
-std::set<std::pair<int, const void*>> g_attr_done;  // (device, kernel) pairs already raised
+std::map<std::pair<int, const void*>, int> g_attr_set;  // (device, kernel) -> limit set so far
 }  // namespace
 
 int ensure_smem_limit(const void* kernel, int bytes) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return GPTQ_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_attr_mu);
-  if (g_attr_done.count({dev, kernel})) return GPTQ_OK;
+  auto it = g_attr_set.find({dev, kernel});
+  if (it != g_attr_set.end() && it->second >= bytes) return GPTQ_OK;  // already high enough
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) {
     cudaGetLastError();
     return GPTQ_ERR_CUDA;
   }
-  g_attr_done.insert({dev, kernel});
+  g_attr_set[{dev, kernel}] = bytes;
   return GPTQ_OK;
 }
 

@@ -1,0 +1,561 @@
+// Linear layer on GPTQ-quantized weights: Y = X * W_hat^T with 16-bit activations.
+//
+// Source: the inference side that the pages benchmark on the quantized checkpoints — the
+// "gptq" skill card's kernel-backend section (ExLlama / Marlin / CUDA kernels run 4-bit
+// weights against fp16 activations) and "第5章 GPTQ 实战" §5.2 (generation speed of the
+// quantized model).  The weights come in the checkpoint form of export.cu: qweight
+// [K*bits/32, N] int32 (codes along K, LSB first), qzeros [G, N*bits/32] int32 (zero points
+// along N, LSB first), scales [G, N] fp16, g_idx [K] int32 (any order, so act-order
+// checkpoints work), and
+//     W_hat[n, k] = scales[g_idx[k], n] * (code[k, n] - zero[g_idx[k], n]).
+// The product is defined as Y = X * round16(W_hat)^T: every dequantized weight is rounded
+// once (nearest even) to the activations' 16-bit type, as a 16-bit tensor-core operand
+// is, and products are accumulated in fp32.  scale * (code - zero) is exact in fp32 (an
+// 11-bit scale times an integer below 2^8), so round16 sees the exact value.
+//
+// Two regimes:
+// * decode (M <= 4 rows of X): HBM-bound on the packed weights.  gemv_kernel streams the
+//   weights once (16-byte loads, coalesced along N), dequantizes in registers and
+//   accumulates on the CUDA cores, split over K across CTAs; a second pass adds the K
+//   splits in a fixed order (deterministic).
+// * prefill / calibration (M > 4): the weights are dequantized once into a 16-bit [N, K]
+//   matrix (dequant_kernel, HBM-bound), and gemm_tn_kernel multiplies on the 5th-generation
+//   tensor cores: TMA loads of both K-major operands with 128-byte swizzle into a 4-stage
+//   ring, tcgen05.mma kind::f16 into a TMEM accumulator of 128 x 256, persistent CTAs with
+//   two accumulators in TMEM so that one tile's epilogue overlaps the next tile's MMAs.
+#include <cuda.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace gptq {
+namespace {
+
+using namespace sm100;
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float v);
+template <>
+__device__ __forceinline__ __half from_f32<__half>(float v) { return __float2half_rn(v); }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+
+// round16(s * (q - z)) as a float, for 16-bit type T
+template <typename T>
+__device__ __forceinline__ float dq(float s, int q, int z) {
+  return to_f32<T>(from_f32<T>(s * static_cast<float>(q - z)));
+}
+
+__device__ __forceinline__ int clamp_group(int g, int G) { return g < 0 ? 0 : (g >= G ? G - 1 : g); }
+
+// ------------------------------------------------------------------ dequantization
+// One CTA per 64 (k) x 64 (n) tile: dequantize into shared memory (reads coalesced along n),
+// then write rows of W [N, K] (128 contiguous bytes per n, coalesced along k).
+constexpr int DQ_T = 64;
+template <int BITS, typename T>
+__global__ void __launch_bounds__(256) dequant_kernel(const int32_t* __restrict__ qweight,
+                                                      const int32_t* __restrict__ qzeros,
+                                                      const __half* __restrict__ scales,
+                                                      const int32_t* __restrict__ g_idx, int G, int64_t K,
+                                                      int64_t N, T* __restrict__ W) {
+  __shared__ __align__(16) T tile[DQ_T][DQ_T + 8];
+  constexpr int FPW = 32 / BITS;
+  constexpr uint32_t MASK = (1u << BITS) - 1u;
+  const int64_t k0 = static_cast<int64_t>(blockIdx.x) * DQ_T, n0 = static_cast<int64_t>(blockIdx.y) * DQ_T;
+  const int t = threadIdx.x;
+  const int nl = t % DQ_T;
+  const int kq = (t / DQ_T) * 16;  // 16 consecutive k per thread
+  const int64_t n = n0 + nl;
+  const int64_t zw = N * BITS / 32;
+  if (n < N) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int64_t k = k0 + kq + i;
+      float v = 0.f;
+      if (k < K) {
+        if (i == 0 || (k % FPW) == 0) word = static_cast<uint32_t>(__ldg(qweight + (k / FPW) * N + n));
+        const int q = static_cast<int>((word >> ((k % FPW) * BITS)) & MASK);
+        const int g = clamp_group(__ldg(g_idx + k), G);
+        const float s = __half2float(__ldg(scales + static_cast<int64_t>(g) * N + n));
+        const uint32_t zword = static_cast<uint32_t>(__ldg(qzeros + static_cast<int64_t>(g) * zw + (n * BITS) / 32));
+        const int z = static_cast<int>((zword >> ((n * BITS) % 32)) & MASK);
+        v = dq<T>(s, q, z);
+      }
+      tile[nl][kq + i] = from_f32<T>(v);
+    }
+  }
+  __syncthreads();
+  // 64 rows x 8 chunks of 16 bytes
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int e = t + 256 * r;
+    const int row = e / 8, ch = e % 8;
+    const int64_t nn = n0 + row, kk = k0 + ch * 8;
+    if (nn < N && kk < K)  // K % 8 == 0: a chunk is wholly inside or outside
+      *reinterpret_cast<uint4*>(W + nn * K + kk) = *reinterpret_cast<const uint4*>(&tile[row][ch * 8]);
+  }
+}
+
+// ------------------------------------------------------------------ tcgen05 GEMM, both operands K-major
+constexpr int GBM = 128;  // rows of X per tile = UMMA M
+constexpr int GBN = 256;  // output columns per tile = UMMA N
+constexpr int GBK = 64;   // K per stage: one 128-byte swizzle row
+constexpr int GSTAGES = 4;
+constexpr int GA_BYTES = GBM * GBK * 2;
+constexpr int GB_BYTES = GBN * GBK * 2;
+constexpr int GSTAGE_BYTES = GA_BYTES + GB_BYTES;  // 48 KiB
+constexpr int GTHREADS = 320;
+constexpr int GSMEM = GSTAGES * GSTAGE_BYTES + 1024 + 256;
+constexpr uint32_t GWAIT = 1u << 24;
+
+__device__ int g_gemm_status = 0;
+
+// K-major operand, 128-byte swizzle: rows of 64 16-bit elements (128 bytes), 8-row atoms of
+// 1024 bytes (stride-dimension offset); the leading-dimension offset is unused because one
+// MMA's K (16 elements, 32 bytes) lies inside a swizzle row.  K steps inside the row
+// advance the start address by 32 bytes.
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t saddr) { return smem_desc_sw128(saddr, 16, 1024); }
+
+template <uint32_t FMT, typename TOut>
+__global__ void __launch_bounds__(GTHREADS, 1)
+    gemm_tn_kernel(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb,
+                   TOut* __restrict__ Y, int M, int N, int K, int mt, int nt) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + GSTAGES * GSTAGE_BYTES);
+  uint64_t* empty = full + GSTAGES;
+  uint64_t* accf = empty + GSTAGES;
+  uint64_t* acce = accf + 2;
+  uint64_t* done = acce + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = static_cast<int>(gridDim.x);
+  const int units = mt * nt;
+  const int nk = (K + GBK - 1) / GBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < GSTAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accf[b], 1);
+      mbar_init(&acce[b], 8);
+    }
+    mbar_init(done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  bool ok = true;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer
+      tma_prefetch_desc(&ta);
+      tma_prefetch_desc(&tb);
+      int stage = 0, issued = 0;
+      uint32_t ph = 0;
+      for (int u = blockIdx.x; u < units && ok; u += G) {
+        const int m0 = (u / nt) * GBM, n0 = (u % nt) * GBN;
+        for (int ks = 0; ks < nk; ++ks) {
+          if (!mbar_wait(&empty[stage], ph ^ 1u, GWAIT)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * GSTAGE_BYTES;
+          mbar_arrive_expect_tx(&full[stage], GSTAGE_BYTES);
+          tma_load_2d(sa, &ta, &full[stage], ks * GBK, m0);
+          tma_load_2d(sa + GA_BYTES, &tb, &full[stage], ks * GBK, n0);
+          ++issued;
+          if (++stage == GSTAGES) {
+            stage = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      // no copy of ours may still be landing in shared memory when the CTA leaves
+      for (int k = 0; k < min(issued, GSTAGES); ++k) {
+        int s = stage - 1 - k;
+        uint32_t p = ph;
+        while (s < 0) {
+          s += GSTAGES;
+          p ^= 1u;
+        }
+        mbar_wait(&full[s], p, GWAIT);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- UMMA issuer
+      constexpr uint32_t idesc = instr_desc(FMT, false, false, GBM, GBN);
+      int stage = 0, cg = 0;
+      uint32_t ph = 0;
+      for (int u = blockIdx.x; u < units && ok; u += G, ++cg) {
+        const int b = cg & 1;
+        if (!mbar_wait(&acce[b], ((cg >> 1) & 1) ^ 1u, GWAIT)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t dcol = tmem + static_cast<uint32_t>(b * GBN);
+        for (int ks = 0; ks < nk; ++ks) {
+          if (!mbar_wait(&full[stage], ph, GWAIT)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * GSTAGE_BYTES);
+          const uint32_t sb = sa + GA_BYTES;
+#pragma unroll
+          for (int k = 0; k < GBK / 16; ++k)
+            umma_f16(dcol, kmajor_desc(sa + k * 32), kmajor_desc(sb + k * 32), idesc, (ks > 0 || k > 0) ? 1u : 0u);
+          umma_commit(&empty[stage]);
+          if (++stage == GSTAGES) {
+            stage = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;  // an incomplete accumulator is never handed to the epilogue
+        umma_commit(&accf[b]);
+      }
+      umma_commit(done);
+      mbar_wait(done, 0, GWAIT);
+    }
+  } else {
+    // ---------------- epilogue (warps 2..9): TMEM -> registers -> 16-bit Y
+    const int quad = warp & 3;         // TMEM lane quarter of this warp
+    const int half = (warp - 2) >> 2;  // which 128 of the 256 columns
+    int cg = 0;
+    for (int u = blockIdx.x; u < units; u += G, ++cg) {
+      const int b = cg & 1;
+      if (!mbar_wait(&accf[b], (cg >> 1) & 1, GWAIT)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int m = (u / nt) * GBM + quad * 32 + lane;
+      const int nb = (u % nt) * GBN + half * 128;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float v[32];
+        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quad * 32) << 16) +
+                               static_cast<uint32_t>(b * GBN + half * 128 + q * 32),
+                           v);
+        if (m < M) {
+          TOut* yrow = Y + static_cast<int64_t>(m) * N;
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) {
+            const int n = nb + q * 32 + c8 * 8;
+            if (n < N) {  // N % 8 == 0: an 8-column chunk is wholly inside or outside
+              alignas(16) TOut o[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) o[e] = from_f32<TOut>(v[c8 * 8 + e]);
+              *reinterpret_cast<uint4*>(yrow + n) = *reinterpret_cast<const uint4*>(o);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acce[b]);
+    }
+  }
+  if (!ok) atomicExch(&g_gemm_status, kStatusTimeout);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ decode GEMV (M <= 4)
+constexpr int GV_THREADS = 256;  // 8 warps; a lane owns 4 consecutive outputs
+constexpr int GV_N = 128;        // outputs per CTA
+constexpr int GV_MAXM = 4;
+
+template <int BITS, typename T>
+__global__ void __launch_bounds__(GV_THREADS) gemv_kernel(const T* __restrict__ X, int M, int64_t K,
+                                                          const int32_t* __restrict__ qweight,
+                                                          const int32_t* __restrict__ qzeros,
+                                                          const __half* __restrict__ scales,
+                                                          const int32_t* __restrict__ g_idx, int G, int64_t N,
+                                                          int kchunk, float* __restrict__ partial) {
+  constexpr int FPW = 32 / BITS;
+  constexpr uint32_t MASK = (1u << BITS) - 1u;
+  extern __shared__ __align__(16) float gsm[];
+  float* xs = gsm;                                     // [GV_MAXM][kchunk]
+  int* gs = reinterpret_cast<int*>(xs + GV_MAXM * kchunk);  // [kchunk]
+  float* red = reinterpret_cast<float*>(gs + kchunk);  // [8][GV_MAXM][GV_N]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t klo = static_cast<int64_t>(blockIdx.y) * kchunk;
+  const int kn = static_cast<int>(min(static_cast<int64_t>(kchunk), K - klo));
+  for (int e = tid; e < kn; e += GV_THREADS) {
+    gs[e] = clamp_group(__ldg(g_idx + klo + e), G);
+#pragma unroll
+    for (int m = 0; m < GV_MAXM; ++m) xs[m * kchunk + e] = m < M ? to_f32<T>(X[m * K + klo + e]) : 0.f;
+  }
+  __syncthreads();
+  const int64_t n = static_cast<int64_t>(blockIdx.x) * GV_N + lane * 4;
+  float acc[GV_MAXM][4];
+#pragma unroll
+  for (int m = 0; m < GV_MAXM; ++m)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[m][j] = 0.f;
+  if (n < N) {
+    const int64_t zw = N * BITS / 32;
+    const int zshift = static_cast<int>((n * BITS) % 32);
+    const int rows = kn / FPW;  // kchunk and K are multiples of FPW
+    int gcur = -1;
+    float s[4];
+    int z[4];
+    for (int r = warp; r < rows; r += 8) {
+      const int64_t wrow = klo / FPW + r;
+      const int4 w4 = __ldg(reinterpret_cast<const int4*>(qweight + wrow * N + n));
+      const uint32_t wv[4] = {static_cast<uint32_t>(w4.x), static_cast<uint32_t>(w4.y), static_cast<uint32_t>(w4.z),
+                              static_cast<uint32_t>(w4.w)};
+#pragma unroll
+      for (int f = 0; f < FPW; ++f) {
+        const int kl = r * FPW + f;
+        const int g = gs[kl];
+        if (g != gcur) {
+          gcur = g;
+          const uint2 s4 = __ldg(reinterpret_cast<const uint2*>(scales + static_cast<int64_t>(g) * N + n));
+          const __half2 s01 = *reinterpret_cast<const __half2*>(&s4.x);
+          const __half2 s23 = *reinterpret_cast<const __half2*>(&s4.y);
+          s[0] = __low2float(s01);
+          s[1] = __high2float(s01);
+          s[2] = __low2float(s23);
+          s[3] = __high2float(s23);
+          const uint32_t zword = static_cast<uint32_t>(__ldg(qzeros + static_cast<int64_t>(g) * zw + (n * BITS) / 32));
+#pragma unroll
+          for (int j = 0; j < 4; ++j) z[j] = static_cast<int>((zword >> (zshift + j * BITS)) & MASK);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float w = dq<T>(s[j], static_cast<int>((wv[j] >> (f * BITS)) & MASK), z[j]);
+#pragma unroll
+          for (int m = 0; m < GV_MAXM; ++m) acc[m][j] = fmaf(xs[m * kchunk + kl], w, acc[m][j]);
+        }
+      }
+    }
+  }
+  // the 8 warps' partial sums of this CTA's outputs, added in a fixed order
+#pragma unroll
+  for (int m = 0; m < GV_MAXM; ++m)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) red[(warp * GV_MAXM + m) * GV_N + lane * 4 + j] = acc[m][j];
+  __syncthreads();
+  for (int e = tid; e < GV_MAXM * GV_N; e += GV_THREADS) {
+    const int m = e / GV_N, c = e % GV_N;
+    const int64_t nn = static_cast<int64_t>(blockIdx.x) * GV_N + c;
+    if (m < M && nn < N) {
+      float t = 0.f;
+      for (int w = 0; w < 8; ++w) t += red[(w * GV_MAXM + m) * GV_N + c];
+      partial[(static_cast<int64_t>(blockIdx.y) * M + m) * N + nn] = t;
+    }
+  }
+}
+
+// Y[m, n] = sum over K splits of partial[s, m, n], in split order.
+template <typename T>
+__global__ void split_sum_kernel(const float* __restrict__ partial, int S, int M, int64_t N, T* __restrict__ Y) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= static_cast<int64_t>(M) * N) return;
+  float t = 0.f;
+  for (int s = 0; s < S; ++s) t += partial[static_cast<int64_t>(s) * M * N + i];
+  Y[i] = from_f32<T>(t);
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<EncodeTiledFn>(p);
+    return static_cast<EncodeTiledFn>(nullptr);
+  }();
+  return fn;
+}
+
+// rows x K (K contiguous) 16-bit matrix, boxes of 64 (K) x box_rows, 128-byte swizzle
+int kmajor_map(CUtensorMap* tm, const void* base, int bf16, int64_t rows, int64_t K, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return GPTQ_ERR_CUDA;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+  cuuint32_t box[2] = {GBK, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(tm, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                         const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? GPTQ_OK : GPTQ_ERR_CUDA;
+}
+
+template <uint32_t FMT, typename T>
+int launch_gemm(const T* X, const T* Wd, T* Y, int64_t M, int64_t N, int64_t K, cudaStream_t s) {
+  GPTQ_TRY(ensure_smem_limit(reinterpret_cast<const void*>(gemm_tn_kernel<FMT, T>), GSMEM));
+  CUtensorMap ta, tb;
+  GPTQ_TRY(kmajor_map(&ta, X, FMT == 1, M, K, GBM));
+  GPTQ_TRY(kmajor_map(&tb, Wd, FMT == 1, N, K, GBN));
+  const int64_t mt = (M + GBM - 1) / GBM, nt = (N + GBN - 1) / GBN;
+  if (mt * nt >= (int64_t(1) << 31)) return GPTQ_ERR_UNSUPPORTED;
+  const int grid = static_cast<int>(std::min<int64_t>(num_sms(), mt * nt));
+  gemm_tn_kernel<FMT, T><<<grid, GTHREADS, GSMEM, s>>>(ta, tb, Y, static_cast<int>(M), static_cast<int>(N),
+                                                       static_cast<int>(K), static_cast<int>(mt), static_cast<int>(nt));
+  return after_launch();
+}
+
+template <int BITS, typename T>
+int launch_dequant(const int32_t* qweight, const int32_t* qzeros, const __half* scales, const int32_t* g_idx, int G,
+                   int64_t K, int64_t N, T* W, cudaStream_t s) {
+  const dim3 grid(static_cast<unsigned>((K + DQ_T - 1) / DQ_T), static_cast<unsigned>((N + DQ_T - 1) / DQ_T));
+  dequant_kernel<BITS, T><<<grid, 256, 0, s>>>(qweight, qzeros, scales, g_idx, G, K, N, W);
+  return after_launch();
+}
+
+template <typename T>
+int dequant_any(int bits, const int32_t* qw, const int32_t* qz, const __half* sc, const int32_t* gi, int G, int64_t K,
+                int64_t N, T* W, cudaStream_t s) {
+  if (bits == 2) return launch_dequant<2, T>(qw, qz, sc, gi, G, K, N, W, s);
+  if (bits == 4) return launch_dequant<4, T>(qw, qz, sc, gi, G, K, N, W, s);
+  return launch_dequant<8, T>(qw, qz, sc, gi, G, K, N, W, s);
+}
+
+template <int BITS, typename T>
+int launch_gemv(const T* X, int M, int64_t K, const int32_t* qw, const int32_t* qz, const __half* sc,
+                const int32_t* gi, int G, int64_t N, T* Y, cudaStream_t s) {
+  // K split so that about four CTAs per SM stream the weights; every split a multiple of
+  // 64 columns (whole words for every bit width).
+  const int64_t nblk = (N + GV_N - 1) / GV_N;
+  int64_t S = std::max<int64_t>(1, (4 * num_sms() + nblk - 1) / nblk);
+  int64_t kchunk = std::max<int64_t>(64, (((K + S - 1) / S) + 63) / 64 * 64);
+  kchunk = std::min<int64_t>(kchunk, 4096);
+  S = (K + kchunk - 1) / kchunk;
+  if (S > 65535) return GPTQ_ERR_UNSUPPORTED;
+  const size_t smem = (GV_MAXM * kchunk + kchunk) * 4 + 8 * GV_MAXM * GV_N * 4;
+  GPTQ_TRY(ensure_smem_limit(reinterpret_cast<const void*>(gemv_kernel<BITS, T>), static_cast<int>(smem)));
+  float* partial = nullptr;
+  GPTQ_TRY(pool_alloc(reinterpret_cast<void**>(&partial), static_cast<size_t>(S) * M * N * 4, s));
+  gemv_kernel<BITS, T><<<dim3(static_cast<unsigned>(nblk), static_cast<unsigned>(S)), GV_THREADS, smem, s>>>(
+      X, M, K, qw, qz, sc, gi, G, N, static_cast<int>(kchunk), partial);
+  int st = after_launch();
+  if (st == GPTQ_OK) {
+    const int64_t cnt = static_cast<int64_t>(M) * N;
+    split_sum_kernel<T><<<static_cast<unsigned>((cnt + 255) / 256), 256, 0, s>>>(partial, static_cast<int>(S), M, N, Y);
+    st = after_launch();
+  }
+  pool_free(partial, s);
+  return st;
+}
+
+template <typename T>
+int gemv_any(int bits, const T* X, int M, int64_t K, const int32_t* qw, const int32_t* qz, const __half* sc,
+             const int32_t* gi, int G, int64_t N, T* Y, cudaStream_t s) {
+  if (bits == 2) return launch_gemv<2, T>(X, M, K, qw, qz, sc, gi, G, N, Y, s);
+  if (bits == 4) return launch_gemv<4, T>(X, M, K, qw, qz, sc, gi, G, N, Y, s);
+  return launch_gemv<8, T>(X, M, K, qw, qz, sc, gi, G, N, Y, s);
+}
+
+int check_qlinear(const int32_t* qweight, const int32_t* qzeros, const uint16_t* scales, const int32_t* g_idx,
+                  int64_t groups, int64_t n_in, int64_t n_out, int bits) {
+  if (!qweight || !qzeros || !scales || !g_idx) return GPTQ_ERR_INVALID_ARG;
+  if (n_in <= 0 || n_out <= 0 || groups <= 0) return GPTQ_ERR_INVALID_ARG;
+  if (bits != 2 && bits != 3 && bits != 4 && bits != 8) return GPTQ_ERR_INVALID_ARG;
+  if (bits == 3) return GPTQ_ERR_UNSUPPORTED;  // fields straddle words; not handled here
+  // whole 32-bit words of zero points per group (n_out * bits % 32), 16-byte output rows
+  if (n_in % 64 != 0 || n_out % 8 != 0 || (n_out * bits) % 32 != 0 || groups > n_in || n_in > (int64_t(1) << 30) ||
+      n_out > (int64_t(1) << 30))
+    return GPTQ_ERR_UNSUPPORTED;
+  if (!aligned16(qweight) || !aligned16(qzeros) || !aligned16(scales) || !aligned16(g_idx)) return GPTQ_ERR_UNSUPPORTED;
+  return GPTQ_OK;
+}
+
+}  // namespace
+
+int gemm_bf16_tn(const void* X, const void* Wd, void* Y, int64_t M, int64_t N, int64_t K, int x_dtype,
+                 cudaStream_t s) {
+  if (x_dtype == GPTQ_BF16)
+    return launch_gemm<1, __nv_bfloat16>(static_cast<const __nv_bfloat16*>(X), static_cast<const __nv_bfloat16*>(Wd),
+                                         static_cast<__nv_bfloat16*>(Y), M, N, K, s);
+  return launch_gemm<0, __half>(static_cast<const __half*>(X), static_cast<const __half*>(Wd), static_cast<__half*>(Y),
+                                M, N, K, s);
+}
+
+int gemm_device_status(int clear) {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_gemm_status, sizeof(int)) != cudaSuccess) return GPTQ_ERR_CUDA;
+  if (clear) {
+    int z = 0;
+    if (cudaMemcpyToSymbol(g_gemm_status, &z, sizeof(int)) != cudaSuccess) return GPTQ_ERR_CUDA;
+  }
+  return v;
+}
+
+}  // namespace gptq
+
+using namespace gptq;
+
+extern "C" int gptq_dequantize_weight(const int32_t* qweight, const int32_t* qzeros, const uint16_t* scales_f16,
+                                      const int32_t* g_idx, int64_t groups, int64_t n_in, int64_t n_out, int bits,
+                                      int out_dtype, void* W, void* stream) {
+  GPTQ_TRY(check_qlinear(qweight, qzeros, scales_f16, g_idx, groups, n_in, n_out, bits));
+  if (!W) return GPTQ_ERR_INVALID_ARG;
+  if (out_dtype != GPTQ_F16 && out_dtype != GPTQ_BF16) return GPTQ_ERR_INVALID_ARG;
+  if (!aligned16(W)) return GPTQ_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const __half* sc = reinterpret_cast<const __half*>(scales_f16);
+  const int G = static_cast<int>(groups);
+  if (out_dtype == GPTQ_BF16)
+    return dequant_any<__nv_bfloat16>(bits, qweight, qzeros, sc, g_idx, G, n_in, n_out, static_cast<__nv_bfloat16*>(W), s);
+  return dequant_any<__half>(bits, qweight, qzeros, sc, g_idx, G, n_in, n_out, static_cast<__half*>(W), s);
+}
+
+extern "C" int gptq_quantized_linear(const void* X, int x_dtype, int64_t M, int64_t n_in, const int32_t* qweight,
+                                     const int32_t* qzeros, const uint16_t* scales_f16, const int32_t* g_idx,
+                                     int64_t groups, int64_t n_out, int bits, void* Y, void* stream) {
+  GPTQ_TRY(check_qlinear(qweight, qzeros, scales_f16, g_idx, groups, n_in, n_out, bits));
+  if (M < 0 || ((!X || !Y) && M > 0)) return GPTQ_ERR_INVALID_ARG;  // no rows: X and Y may be NULL
+  if (x_dtype != GPTQ_F16 && x_dtype != GPTQ_BF16) return GPTQ_ERR_INVALID_ARG;
+  if (M == 0) return GPTQ_OK;
+  if (M >= (int64_t(1) << 31)) return GPTQ_ERR_UNSUPPORTED;
+  if (!aligned16(X) || !aligned16(Y)) return GPTQ_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const __half* sc = reinterpret_cast<const __half*>(scales_f16);
+  const int G = static_cast<int>(groups);
+  if (M <= GV_MAXM) {
+    if (x_dtype == GPTQ_BF16)
+      return gemv_any<__nv_bfloat16>(bits, static_cast<const __nv_bfloat16*>(X), static_cast<int>(M), n_in, qweight,
+                                     qzeros, sc, g_idx, G, n_out, static_cast<__nv_bfloat16*>(Y), s);
+    return gemv_any<__half>(bits, static_cast<const __half*>(X), static_cast<int>(M), n_in, qweight, qzeros, sc, g_idx,
+                            G, n_out, static_cast<__half*>(Y), s);
+  }
+  void* Wd = nullptr;
+  GPTQ_TRY(pool_alloc(&Wd, static_cast<size_t>(n_in) * n_out * 2, s));
+  int st = x_dtype == GPTQ_BF16
+               ? dequant_any<__nv_bfloat16>(bits, qweight, qzeros, sc, g_idx, G, n_in, n_out,
+                                            static_cast<__nv_bfloat16*>(Wd), s)
+               : dequant_any<__half>(bits, qweight, qzeros, sc, g_idx, G, n_in, n_out, static_cast<__half*>(Wd), s);
+  if (st == GPTQ_OK) st = gemm_bf16_tn(X, Wd, Y, M, n_out, n_in, x_dtype, s);
+  pool_free(Wd, s);
+  return st;
+}

@@ -35,6 +35,8 @@ __all__ = [
     "CONFIGS",
     "weight_for",
     "acts_for",
+    "checkpoint_parts",
+    "decoder_layer_inputs",
 ]
 
 MODULE_INDEX = {"q": 0, "k": 1, "v": 2, "o": 3, "gate": 4, "fc1": 4, "up": 5, "down": 6, "fc2": 6}
@@ -132,6 +134,39 @@ class StudentTActs(HeavyChannelActs):
         chi2 = (torch.randn(self.nu, self.n, generator=g, device=device) ** 2).sum(0)
         tau = z / torch.sqrt(chi2 / self.nu)
         return 1.0 + tau.abs()
+
+
+def checkpoint_parts(n_out, n_in, bits, group_size, seed, act_order=False, scale_range=(0.002, 0.02)):
+    """Random parts of a quantized linear (uniform codes and zero points, log-uniform
+    scales rounded to float16, and group indices): codes [n_out, n_in], zeros [G, n_out],
+    scales [G, n_out] float16, g_idx [n_in].  With act_order the groups are runs of
+    group_size columns in a random column order (g_idx not monotone), as desc_act makes
+    them.  Random numbers only; packing is up to the caller."""
+    g = _gen(seed, "cpu")
+    G = 1 if group_size == -1 else n_in // group_size
+    gsz = n_in if group_size == -1 else group_size
+    codes = torch.randint(0, 2 ** bits, (n_out, n_in), generator=g)
+    zeros = torch.randint(0, 2 ** bits, (G, n_out), generator=g)
+    lo, hi = math.log(scale_range[0]), math.log(scale_range[1])
+    scales = torch.exp(lo + (hi - lo) * torch.rand(G, n_out, generator=g)).half()
+    order = torch.randperm(n_in, generator=g) if act_order else torch.arange(n_in)
+    g_idx = torch.empty(n_in, dtype=torch.int32)
+    g_idx[order] = (torch.arange(n_in) // gsz).to(torch.int32)
+    return codes, zeros, scales, g_idx
+
+
+def decoder_layer_inputs(hidden, inter, tokens, seed, dtype=torch.bfloat16):
+    """Calibration hidden states and weights of one synthetic Llama-style decoder layer:
+    h [tokens, hidden] with heavy-tailed channels (the Llama-shaped configs' activation
+    law), the seven linear weights with the outlier law (fp16), and the two norm weights
+    1 + 0.1 N(0, 1).  Random numbers only."""
+    h = StudentTActs(hidden, tokens, seed, dtype=dtype).full()
+    shapes = {"q": (hidden, hidden), "k": (hidden, hidden), "v": (hidden, hidden), "o": (hidden, hidden),
+              "gate": (inter, hidden), "up": (inter, hidden), "down": (hidden, inter)}
+    weights = {name: outlier_weight(no, ni, seed * 10 + MODULE_INDEX[name]) for name, (no, ni) in shapes.items()}
+    g = _gen(seed * 10 + 9, "cpu")
+    gammas = tuple((1.0 + 0.1 * torch.randn(hidden, generator=g)).to(dtype) for _ in range(2))
+    return h, weights, gammas
 
 
 @dataclass

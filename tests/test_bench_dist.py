@@ -55,15 +55,21 @@ def test_reference_arm_two_ranks_prints_one_line():
     assert d["impl"] == "reference" and d["unit"] == "weight-cols/s" and d["value"] > 0
 
 
-def test_hessian_traffic_profile_parses_per_launch():
-    """The bench's roofline takes the Hessian's DRAM traffic per launch from the committed
-    ncu summary: one figure per distinct Hessian of the Llama-2-7B layer, in launch order,
-    each at least the launch's algorithmic bytes (X once + H once)."""
+def test_hessian_traffic_from_small_case_counters(tmp_path, monkeypatch):
+    """The bench's roofline `traffic` comes from committed ncu counters of small-case
+    launches: per width a line through two token counts, evaluated at the layer's T; it is
+    null when the counters belong to another version of the kernel or a width is missing."""
     import bench
     from post_weight_quantization_layer_b200 import synth
 
     cfg = synth.CONFIGS["llama7b"]
-    traffic = bench.load_traffic()
-    assert traffic is not None and len(traffic) == len(cfg.hessian_n)
-    for n, t in zip(cfg.hessian_n, traffic):
-        assert t >= cfg.tokens * n * 2 + n * n * 4
+    f = tmp_path / "traffic.json"
+    caps = [{"n": n, "tokens": t, "dram_bytes": 1000 * n + 3 * t * n} for n in (4096, 11008) for t in (16384, 32768)]
+    f.write_text(json.dumps({"kernel_sha": bench.kernel_source_sha(), "captures": caps}))
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(f))
+    tr = bench.hessian_traffic(cfg, cfg.tokens)
+    assert tr["per_launch"] == [1000 * n + 3 * cfg.tokens * n for n in cfg.hessian_n]
+    f.write_text(json.dumps({"kernel_sha": "other", "captures": caps}))
+    assert bench.hessian_traffic(cfg, cfg.tokens) is None
+    f.write_text(json.dumps({"kernel_sha": bench.kernel_source_sha(), "captures": caps[:2]}))
+    assert bench.hessian_traffic(cfg, cfg.tokens) is None

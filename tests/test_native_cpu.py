@@ -161,3 +161,36 @@ def test_python_binding_rejects_mismatched_tensors():
     for fn, msg in cases:
         with pytest.raises(ValueError, match=msg):
             fn()
+
+
+def test_checkpoint_and_forward_rejections(L):
+    """Host-side rejections of the export, quantized-linear and layer-forward entry points
+    (nothing reaches the GPU)."""
+    ex = L.gptq_export_layer
+    assert ex(None, FAKE, 4, 64, 4, FAKE, FAKE, None) == INVALID
+    assert ex(FAKE, FAKE, 0, 64, 4, FAKE, FAKE, None) == INVALID
+    assert ex(FAKE, FAKE, 4, 64, 5, FAKE, FAKE, None) == INVALID
+    assert ex(FAKE, FAKE, 4, 36, 4, FAKE, FAKE, None) == UNSUPPORTED       # 36*4 % 32
+    assert ex(MISALIGNED, FAKE, 4, 64, 4, FAKE, FAKE, None) == UNSUPPORTED
+    dq = L.gptq_dequantize_weight
+    assert dq(None, FAKE, FAKE, FAKE, 4, 512, 64, 4, 1, FAKE, None) == INVALID
+    assert dq(FAKE, FAKE, FAKE, FAKE, 4, 512, 64, 5, 1, FAKE, None) == INVALID
+    assert dq(FAKE, FAKE, FAKE, FAKE, 4, 512, 64, 3, 1, FAKE, None) == UNSUPPORTED   # 3-bit
+    assert dq(FAKE, FAKE, FAKE, FAKE, 4, 500, 64, 4, 1, FAKE, None) == UNSUPPORTED   # n_in % 64
+    assert dq(FAKE, FAKE, FAKE, FAKE, 4, 512, 72, 2, 1, FAKE, None) == UNSUPPORTED   # 72*2 % 32
+    assert dq(FAKE, FAKE, FAKE, FAKE, 4, 512, 64, 4, 0, FAKE, None) == INVALID       # fp32 output
+    ql = L.gptq_quantized_linear
+    assert ql(FAKE, 2, 8, 512, FAKE, FAKE, FAKE, FAKE, 4, 64, 4, None, None) == INVALID
+    assert ql(FAKE, 0, 8, 512, FAKE, FAKE, FAKE, FAKE, 4, 64, 4, FAKE, None) == INVALID   # fp32 X
+    assert ql(FAKE, 2, -1, 512, FAKE, FAKE, FAKE, FAKE, 4, 64, 4, FAKE, None) == INVALID
+    assert ql(FAKE, 2, 0, 512, FAKE, FAKE, FAKE, FAKE, 4, 64, 4, FAKE, None) == 0         # no rows: no-op
+    assert ql(None, 2, 0, 512, FAKE, FAKE, FAKE, FAKE, 4, 64, 4, None, None) == 0         # ... even with NULL X, Y
+    assert ql(MISALIGNED, 2, 8, 512, FAKE, FAKE, FAKE, FAKE, 4, 64, 4, FAKE, None) == UNSUPPORTED
+    assert L.gptq_rmsnorm(FAKE, 0, 4, 64, FAKE, 1e-6, FAKE, None) == INVALID
+    assert L.gptq_rmsnorm(FAKE, 2, 4, 64, None, 1e-6, FAKE, None) == INVALID
+    assert L.gptq_rope(FAKE, 2, 16, 4, 63, 8, 10000.0, None) == INVALID   # odd head_dim
+    assert L.gptq_attention(FAKE, FAKE, FAKE, 2, 100, 4, 64, 32, FAKE, None) == INVALID  # ragged sequences
+    assert L.gptq_attention(FAKE, FAKE, FAKE, 2, 64, 1, 256, 32, FAKE, None) == UNSUPPORTED  # head_dim > 128
+    assert L.gptq_silu_mul(FAKE, None, 2, 8, FAKE, None) == INVALID
+    assert L.gptq_add(FAKE, FAKE, 1, -1, FAKE, None) == INVALID
+    assert L.gptq_test_wait_expiry(1, 0) == INVALID
