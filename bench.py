@@ -16,8 +16,10 @@ The headline metric is weight columns quantized per second over the layer
 decoder layer.  Multi-GPU runs are independent replicas (one layer per rank,
 weak scaling); ranks only meet at barriers and at the max-over-ranks timing.
 
-`--impl reference` times the float64 CPU oracle on a bounded sample of the same
-workload and reports the same metric (extrapolated per phase by work).
+`--impl reference` times the float64 CPU oracle on the same workload, one bounded
+piece of the layer per step (pieces at the layer's own shapes, each scaled to the layer
+by an exact work ratio), and reports the same metric; `--cpu-full-layer` times the
+oracle on the whole layer once, beside the sample's estimate.
 """
 
 from __future__ import annotations
@@ -35,6 +37,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "GPTQ ms/layer & weight-cols/s; Hessian TFLOPS; per-phase roofline fraction"
+DATASHEET_BF16_DENSE_TFLOPS = 2250.0
 UNIT = "weight-cols/s"
 
 
@@ -49,6 +52,8 @@ def parse_args():
     p.add_argument("--e2e-steps", type=int, default=6)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--cpu-full-layer", action="store_true",
+                   help="time the float64 oracle on the whole layer once (minutes of CPU) beside the sample estimate")
     return p.parse_args()
 
 
@@ -152,6 +157,19 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ workload
+WORKLOADS = {
+    "tiny": "tiny single linear layer GPTQ (64x256, 512 tokens)",
+    "opt125m": "OPT-125m-shaped decoder layer GPTQ (6 linears, 4 Hessians)",
+    "llama7b": "Llama-2-7B-shaped decoder layer GPTQ (7 linears, 4 Hessians)",
+    "sweep": "4096x11008 down_proj-shaped layer GPTQ (1 linear, 1 Hessian)",
+    "llama70b": "Llama-2-70B-shaped decoder layer GPTQ (7 linears, 4 Hessians)",
+}
+
+
+def workload_name(config):
+    return f"{config}: {WORKLOADS.get(config, config)}"
+
+
 def layer_columns(cfg):
     return sum(m.n_in for m in cfg.layers)
 
@@ -255,17 +273,21 @@ def run_native(args, world, rank, local):
         "algorithmic_flops_per_launch": work["hessian_flops"],
         "per_launch_tflops": [round(x, 1) for x in per_launch],
     }
-    traffic = load_traffic() if args.config == "llama7b" and T == cfg.tokens else None
-    if traffic is not None and len(traffic) == len(launch_ms):
+    traffic = hessian_traffic(cfg, T)
+    if traffic is not None:
         # per launch, like `achieved` (the mean over this layer's Hessian launches)
-        roofline["traffic"] = round(statistics.mean(traffic))
-        roofline["traffic_per_launch"] = traffic
-        roofline["traffic_source"] = "ncu dram__bytes_read.sum + dram__bytes_write.sum, " \
-                                     "profiles/hessian_syrk_dram_llama7b_layer.md"
+        roofline["traffic"] = round(statistics.mean(traffic["per_launch"]))
+        roofline["traffic_per_launch"] = traffic["per_launch"]
+        roofline["traffic_source"] = traffic["source"]
+        roofline["algorithmic_bytes_per_launch"] = [2 * T * n + 4 * n * n for n in cfg.hessian_n]
 
     phases = {
         "hessian": {"ms": round(h_ms, 3), "tflops": round(h_tflops, 1),
-                    "frac_of_bf16_sustained": round(h_tflops / peaks["bf16_sus"], 4)},
+                    "frac_of_bf16_sustained": round(h_tflops / peaks["bf16_sus"], 4),
+                    "frac_of_bf16_burst": round(h_tflops / peaks["bf16"], 4),
+                    "frac_of_datasheet_dense_bf16": round(h_tflops / DATASHEET_BF16_DENSE_TFLOPS, 4),
+                    "datasheet_note": "2250 TFLOP/s: NVIDIA's dense (non-sparse) bf16 figure for B200 at its "
+                                      "boost clock, not measured on this part"},
         "factor": {"ms": round(f_ms, 3), "tflops_fp64": round(f_tflops, 2),
                    "frac_of_fp64_peak": round(f_tflops / fp64_peak, 4)},
         "sweep": {"ms": round(s_ms, 3), "tflops_fp64": round(s_tflops, 2),
@@ -291,7 +313,7 @@ def run_native(args, world, rank, local):
         "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16 activations / fp16 weights; fp32 accumulate; fp32+fp64 sweep",
         "data": "synthetic (seeded Student-t activations, Gaussian+outlier weights; no datasets or checkpoints)",
-        "config": {"workload": f"{args.config}: Llama-2-7B-shaped decoder layer GPTQ (7 linears, 4 Hessians)",
+        "config": {"workload": workload_name(args.config),
                    "tokens": T, "bits": cfg.bits, "group_size": cfg.group_size, "desc_act": cfg.desc_act,
                    "static_groups": cfg.static_groups, "damp_percent": cfg.damp_percent,
                    "weight_cols_per_layer": cols, "parallelism": f"replicas x{world}",
@@ -327,18 +349,45 @@ def measure_fp64_peak(dev):
     return 2 * n ** 3 / (best / 1e3) / 1e12
 
 
-def load_traffic():
-    """DRAM bytes (read + write) per Hessian launch of one decoder layer, from the committed
-    ncu summary of the same bench command (profiles/hessian_syrk_dram_llama7b_layer.md)."""
-    path = os.path.join(ROOT, "profiles", "hessian_syrk_dram_llama7b_layer.md")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "hessian_syrk_traffic.json")
+
+
+def hessian_traffic(cfg, T):
+    """DRAM bytes (read + write) of each Hessian launch of the layer at T tokens, from the
+    committed ncu counters of small-case launches of the same kernel (same widths, fewer
+    tokens): for each width the counters of two token counts give bytes = a + b * T
+    (X is streamed once per token segment group, H written a fixed number of times), which
+    is evaluated at T.  None when the file has no capture of a width, or was taken from
+    another build of the kernel than this source (its `kernel_sha` field)."""
     try:
-        with open(path) as f:
-            for ln in f:
-                if ln.startswith("traffic_bytes_per_launch:"):
-                    return [float(x) for x in ln.split(":", 1)[1].strip().strip("[]").split(",")]
-    except OSError:
-        pass
-    return None
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if d.get("kernel_sha") != kernel_source_sha():
+        return None
+    per_launch = []
+    for n in cfg.hessian_n:
+        pts = sorted((c["tokens"], c["dram_bytes"]) for c in d.get("captures", []) if c["n"] == n)
+        if len(pts) < 2:
+            return None
+        (t0, b0), (t1, b1) = pts[0], pts[-1]
+        slope = (b1 - b0) / (t1 - t0)
+        per_launch.append(round(b1 + slope * (T - t1)))
+    caps = ", ".join(f"n={c['n']} T={c['tokens']}" for c in d["captures"])
+    return {"per_launch": per_launch,
+            "source": f"ncu dram__bytes_read.sum + dram__bytes_write.sum of small-case launches ({caps}), "
+                      f"line through two token counts per width evaluated at T={T}; profiles/hessian_syrk_traffic.json"}
+
+
+def kernel_source_sha():
+    """Short hash of the Hessian kernel's sources (the counters belong to this code)."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("hessian.cu", "hessian_sched.cuh", "sm100.cuh"):
+        with open(os.path.join(ROOT, "post_weight_quantization_layer_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
 
 
 def run_e2e(args, cfg, acts, weights, dev, stream, world, Hbuf):
@@ -415,54 +464,97 @@ def run_e2e(args, cfg, acts, weights, dev, stream, world, Hbuf):
 
 
 # ------------------------------------------------------------------ CPU oracle baseline
-def oracle_sample(cfg, T, budget_scale=1.0):
-    """Time the float64 oracle on a bounded sample and extrapolate each phase to the
-    full decoder layer along its cost structure: the Hessian by T*n^2 (a sample of
-    tokens), the factor by n^3 (a smaller Hessian), the sweep by rows (full-width
-    rows of each distinct n_in; rows are independent given the factor).
-    Returns (seconds per layer, description, seconds spent)."""
-    import numpy as np
+SAMPLE_TOKENS = 8192   # one calibration chunk (the streaming unit of the Hessian)
+SAMPLE_ROWS = 256      # output rows swept per linear
 
-    import oracle as O
-    from post_weight_quantization_layer_b200 import synth
 
-    spent = 0.0
-    n0 = cfg.hessian_n[0]
-    ts = max(256, int(1024 * budget_scale))
-    X = synth.acts_for(cfg, 0, tokens=ts).full().double().numpy()
-    t0 = time.perf_counter()
-    H = O.hessian(X)
-    t_h = time.perf_counter() - t0
-    h_scale = sum(T * n * n for n in cfg.hessian_n) / (ts * n0 * n0)
+class OracleSample:
+    """The float64 oracle on a bounded sample of one decoder layer, cut into pieces whose
+    shapes are the layer's own, each with the factor that scales it to the whole layer:
 
-    nf = min(n0, 2048 if budget_scale < 2 else 4096)
-    t0 = time.perf_counter()
-    O.inverse_cholesky_upper(O.dampen(H[:nf, :nf], cfg.damp_percent))
-    t_f = time.perf_counter() - t0
-    f_scale = sum(n ** 3 for n in cfg.hessian_n) / nf ** 3
-    spent += t_h + t_f
+    * Hessian h: 2 X^T X of one 8,192-token chunk at the full width n_h; the oracle's
+      Hessian of T tokens is the sum of T / 8192 such chunk products (scale T / 8192);
+    * factor h: act-order permutation, damping and inverse-Cholesky factor at the full
+      width (scale 1; the chunk Hessian is made positive definite by the damping, and the
+      factor's cost does not depend on its values);
+    * sweep m: the sweep of SAMPLE_ROWS rows of linear m at its full width against that
+      factor (rows are independent given the factor; scale n_out / SAMPLE_ROWS).
 
-    # Sweep: full-width rows per distinct n_in, with a valid upper-triangular factor
-    # (a scaled identity; the sweep's cost does not depend on the factor's values).
-    rows = max(16, int(128 * budget_scale))
-    t_s_total = 0.0
-    parts = []
-    for n_in in sorted({m.n_in for m in cfg.layers}):
-        W = synth.outlier_weight(rows, n_in, 5).double().numpy()
-        U = np.eye(n_in) * 0.5
+    Inputs are drawn and prepared once (untimed).  `time_piece` times one piece."""
+
+    def __init__(self, cfg, T):
+        import numpy as np
+
+        import oracle as O
+        from post_weight_quantization_layer_b200 import synth
+        self.O, self.np, self.cfg, self.T = O, np, cfg, T
+        self.X = {h: synth.acts_for(cfg, h, tokens=SAMPLE_TOKENS).full().double().numpy()
+                  for h in range(len(cfg.hessian_n))}
+        self.W = {}
+        for m in cfg.layers:
+            W = synth.weight_for(cfg, m).double().numpy()
+            self.W[m.name] = np.ascontiguousarray(W[:SAMPLE_ROWS])
+        self.H, self.factor = {}, {}
+        self.pieces = [("hessian", h) for h in self.X] + [("factor", h) for h in self.X] + \
+                      [("sweep", m.name) for m in cfg.layers]
+        self.times = {p: [] for p in self.pieces}
+
+    def scale(self, piece):
+        kind, key = piece
+        if kind == "hessian":
+            return self.T / SAMPLE_TOKENS
+        if kind == "factor":
+            return 1.0
+        m = next(m for m in self.cfg.layers if m.name == key)
+        return m.n_out / min(SAMPLE_ROWS, m.n_out)
+
+    def _run(self, piece):
+        O, np, cfg = self.O, self.np, self.cfg
+        kind, key = piece
+        if kind == "hessian":
+            self.H[key] = O.hessian(self.X[key])
+        elif kind == "factor":
+            H = self.H[key]
+            perm = O.act_order_perm(H) if cfg.desc_act else np.arange(H.shape[0])
+            U = O.inverse_cholesky_upper(O.dampen(H[np.ix_(perm, perm)], cfg.damp_percent))
+            self.factor[key] = (perm, U)
+        else:
+            m = next(m for m in cfg.layers if m.name == key)
+            perm, U = self.factor[m.h_index]
+            W = self.W[key]
+            O.gptq_sweep(W[:, perm], U, cfg.bits, cfg.sym, cfg.group_size, perm, cfg.static_groups, W,
+                         cfg.blocksize)
+
+    def time_piece(self, piece):
+        """Run one piece (its inputs must exist: Hessian before factor before sweep)."""
         t0 = time.perf_counter()
-        O.gptq_sweep(W, U, cfg.bits, cfg.sym, cfg.group_size, np.arange(n_in), cfg.static_groups, W,
-                     cfg.blocksize)
+        self._run(piece)
         dt = time.perf_counter() - t0
-        spent += dt
-        total_rows = sum(m.n_out for m in cfg.layers if m.n_in == n_in)
-        t_s_total += dt * total_rows / rows
-        parts.append(f"{rows}x{n_in} in {dt:.2f} s (x{total_rows / rows:.0f} rows)")
-    total = t_h * h_scale + t_f * f_scale + t_s_total
-    desc = (f"oracle float64 on host cores: Hessian of {ts} tokens x {n0} in {t_h:.2f} s (x{h_scale:.0f} by T*n^2), "
-            f"factor n={nf} in {t_f:.2f} s (x{f_scale:.1f} by n^3), sweep " + ", ".join(parts) +
-            f"; sample {spent:.1f} s of CPU work")
-    return total, desc, spent
+        self.times[piece].append(dt)
+        return dt
+
+    def run_all(self):
+        """Every piece once, in dependency order (the cpu_baseline measurement)."""
+        for p in self.pieces:
+            self.time_piece(p)
+
+    def layer_seconds(self):
+        """Whole-layer oracle seconds from the mean time of each piece times its scale."""
+        return sum(statistics.mean(self.times[p]) * self.scale(p) for p in self.pieces if self.times[p])
+
+    def spent(self):
+        return sum(sum(v) for v in self.times.values())
+
+    def describe(self):
+        parts = {"hessian": [], "factor": [], "sweep": []}
+        for p in self.pieces:
+            if self.times[p]:
+                parts[p[0]].append(f"{p[1]} {statistics.mean(self.times[p]):.2f} s x{self.scale(p):.4g}")
+        return (f"float64 oracle on the host cores, pieces of the layer at its own shapes, each timed and "
+                f"scaled to the layer: Hessian of one {SAMPLE_TOKENS}-token chunk per input (scale T/{SAMPLE_TOKENS}): "
+                + ", ".join(parts["hessian"]) + "; factor at full width per input: " + ", ".join(parts["factor"]) +
+                f"; sweep of {SAMPLE_ROWS} rows per linear at full width (scale n_out/{SAMPLE_ROWS}): "
+                + ", ".join(parts["sweep"]) + f"; {self.spent():.1f} s of CPU work timed")
 
 
 def cpu_cores():
@@ -475,44 +567,107 @@ def cpu_cores():
 
 
 def cpu_baseline(cfg, T):
-    total, desc, _ = oracle_sample(cfg, T, 4.0)
+    smp = OracleSample(cfg, T)
+    smp.run_all()
+    total = smp.layer_seconds()
     return {"value": round(layer_columns(cfg) / total, 3), "unit": UNIT, "cores": cpu_cores(),
-            "kind": "oracle", "sample": desc, "s_per_layer_extrapolated": round(total, 1)}
+            "kind": "oracle", "sample": smp.describe(), "s_per_layer_extrapolated": round(total, 1)}
 
 
 def run_reference(args, world, rank):
-    """The oracle as the reference arm: rank 0 alone, each step a bounded sample."""
+    """The oracle as the reference arm: rank 0 alone.  Each step is one piece of the layer
+    sample (OracleSample), taken round-robin, so a step is a bounded amount of CPU work;
+    ms_per_step is the time the steps actually took, and the layer-time estimate comes
+    from the per-piece times scaled to the layer (any piece no timed step reached is
+    taken from the set-up pass, which times every piece once)."""
     if rank != 0:
         return None
     from post_weight_quantization_layer_b200 import synth
     cfg = synth.CONFIGS[args.config]
     T = args.tokens or cfg.tokens
+    smp = OracleSample(cfg, T)
+    smp.run_all()  # set-up: every piece's inputs and one timing of each
+    setup = {p: list(v) for p, v in smp.times.items()}
+    for p in smp.pieces:
+        smp.times[p] = []
+    k = 0
     for _ in range(max(args.warmup, 0)):
-        oracle_sample(cfg, T, 0.5)
-    tot = []
-    desc = ""
+        smp._run(smp.pieces[k % len(smp.pieces)])
+        k += 1
+    step_s = []
     for _ in range(args.steps):
-        t, desc, _ = oracle_sample(cfg, T, 0.5)
-        tot.append(t)
-    s = statistics.mean(tot)
-    value = layer_columns(cfg) / s
+        step_s.append(smp.time_piece(smp.pieces[k % len(smp.pieces)]))
+        k += 1
+    for p in smp.pieces:
+        if not smp.times[p]:
+            smp.times[p] = setup[p]
+    layer_s = smp.layer_seconds()
+    value = layer_columns(cfg) / layer_s
+    ms = 1e3 * statistics.mean(step_s) if step_s else 0.0
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": 1,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * s, 1), "higher_is_better": True,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 1), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{args.config}: Llama-2-7B-shaped decoder layer GPTQ (7 linears, 4 Hessians)",
+        "config": {"workload": workload_name(args.config),
                    "tokens": T},
+        "step_is": "one piece of the oracle's layer sample (round-robin over "
+                   f"{len(smp.pieces)} pieces); ms_per_step is measured",
+        "s_per_layer_extrapolated": round(layer_s, 1),
         "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
-                         "sample": desc},
+                         "sample": smp.describe()},
         "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
+
+
+def run_cpu_full_layer(args):
+    """Calibration of the sample: the oracle on the WHOLE decoder layer once (all tokens,
+    all rows; several minutes of CPU), next to the sample's estimate in the same run."""
+    import numpy as np
+
+    import oracle as O
+    from post_weight_quantization_layer_b200 import synth
+    cfg = synth.CONFIGS[args.config]
+    T = args.tokens or cfg.tokens
+    smp = OracleSample(cfg, T)
+    smp.run_all()
+    est = smp.layer_seconds()
+    del smp
+    phase = {"hessian": 0.0, "factor": 0.0, "sweep": 0.0}
+    factors = {}
+    for h, n in enumerate(cfg.hessian_n):
+        acts = synth.acts_for(cfg, h, tokens=T)
+        H = np.zeros((n, n))
+        for i in range(acts.n_chunks):
+            X = acts.get_chunk(i).double().numpy()
+            t0 = time.perf_counter()
+            H += O.hessian(X)
+            phase["hessian"] += time.perf_counter() - t0
+        t0 = time.perf_counter()
+        perm = O.act_order_perm(H) if cfg.desc_act else np.arange(n)
+        U = O.inverse_cholesky_upper(O.dampen(H[np.ix_(perm, perm)], cfg.damp_percent))
+        phase["factor"] += time.perf_counter() - t0
+        factors[h] = (perm, U)
+        del H
+    for m in cfg.layers:
+        W = synth.weight_for(cfg, m).double().numpy()
+        perm, U = factors[m.h_index]
+        t0 = time.perf_counter()
+        O.gptq_sweep(W[:, perm], U, cfg.bits, cfg.sym, cfg.group_size, perm, cfg.static_groups, W, cfg.blocksize)
+        phase["sweep"] += time.perf_counter() - t0
+    full = sum(phase.values())
+    return {"impl": "oracle-full-layer", "config": args.config, "tokens": T, "cores": cpu_cores(),
+            "s_per_layer_measured": round(full, 1), "phases_s": {k: round(v, 1) for k, v in phase.items()},
+            "value_measured": round(layer_columns(cfg) / full, 3), "unit": UNIT,
+            "s_per_layer_sample_estimate": round(est, 1), "estimate_over_measured": round(est / full, 3)}
 
 
 def main():
     args = parse_args()
     world, rank, local = dist_setup(args.gpus)
     try:
-        if args.impl == "reference":
+        if args.cpu_full_layer:
+            line = run_cpu_full_layer(args) if rank == 0 else None
+        elif args.impl == "reference":
             line = run_reference(args, world, rank)
         else:
             line = run_native(args, world, rank, local)
