@@ -464,8 +464,8 @@ def run_e2e(args, cfg, acts, weights, dev, stream, world, Hbuf):
 
 
 # ------------------------------------------------------------------ CPU oracle baseline
-SAMPLE_TOKENS = 8192   # one calibration chunk (the streaming unit of the Hessian)
-SAMPLE_ROWS = 256      # output rows swept per linear
+SAMPLE_TOKENS = 8192           # one calibration chunk (the streaming unit of the Hessian)
+SAMPLE_SWEEP_BYTES = 64 << 20  # fp64 running weights per sampled sweep: out of cache, like the layer's
 
 
 class OracleSample:
@@ -477,8 +477,11 @@ class OracleSample:
     * factor h: act-order permutation, damping and inverse-Cholesky factor at the full
       width (scale 1; the chunk Hessian is made positive definite by the damping, and the
       factor's cost does not depend on its values);
-    * sweep m: the sweep of SAMPLE_ROWS rows of linear m at its full width against that
-      factor (rows are independent given the factor; scale n_out / SAMPLE_ROWS).
+    * sweep of each distinct linear shape (n_out, n_in): rows of its first linear at the
+      full width against that linear's factor, as many rows as make 64 MB of fp64 running
+      weights (a working set out of the host's caches, as the whole layer's is; smaller
+      samples ran up to 1.8x faster per row); rows are independent given the factor and the
+      sweep's time is linear in them (scale: linears of that shape x n_out / rows).
 
     Inputs are drawn and prepared once (untimed).  `time_piece` times one piece."""
 
@@ -490,13 +493,19 @@ class OracleSample:
         self.O, self.np, self.cfg, self.T = O, np, cfg, T
         self.X = {h: synth.acts_for(cfg, h, tokens=SAMPLE_TOKENS).full().double().numpy()
                   for h in range(len(cfg.hessian_n))}
-        self.W = {}
+        self.W, self.rows, self.count = {}, {}, {}
         for m in cfg.layers:
+            shape = (m.n_out, m.n_in)
+            self.count[shape] = self.count.get(shape, 0) + 1
+            if any((o.n_out, o.n_in) == shape for o in cfg.layers[:cfg.layers.index(m)]):
+                continue  # one piece per distinct shape: its first linear
+            rows = min(m.n_out, max(1, SAMPLE_SWEEP_BYTES // (8 * m.n_in)))
             W = synth.weight_for(cfg, m).double().numpy()
-            self.W[m.name] = np.ascontiguousarray(W[:SAMPLE_ROWS])
+            self.W[m.name] = np.ascontiguousarray(W[:rows])
+            self.rows[m.name] = rows
         self.H, self.factor = {}, {}
         self.pieces = [("hessian", h) for h in self.X] + [("factor", h) for h in self.X] + \
-                      [("sweep", m.name) for m in cfg.layers]
+                      [("sweep", name) for name in self.W]
         self.times = {p: [] for p in self.pieces}
 
     def scale(self, piece):
@@ -506,7 +515,7 @@ class OracleSample:
         if kind == "factor":
             return 1.0
         m = next(m for m in self.cfg.layers if m.name == key)
-        return m.n_out / min(SAMPLE_ROWS, m.n_out)
+        return self.count[(m.n_out, m.n_in)] * m.n_out / self.rows[key]
 
     def _run(self, piece):
         O, np, cfg = self.O, self.np, self.cfg
@@ -549,12 +558,14 @@ class OracleSample:
         parts = {"hessian": [], "factor": [], "sweep": []}
         for p in self.pieces:
             if self.times[p]:
-                parts[p[0]].append(f"{p[1]} {statistics.mean(self.times[p]):.2f} s x{self.scale(p):.4g}")
+                rows = f" ({self.rows[p[1]]} rows)" if p[0] == "sweep" else ""
+                parts[p[0]].append(f"{p[1]}{rows} {statistics.mean(self.times[p]):.2f} s x{self.scale(p):.4g}")
         return (f"float64 oracle on the host cores, pieces of the layer at its own shapes, each timed and "
                 f"scaled to the layer: Hessian of one {SAMPLE_TOKENS}-token chunk per input (scale T/{SAMPLE_TOKENS}): "
                 + ", ".join(parts["hessian"]) + "; factor at full width per input: " + ", ".join(parts["factor"]) +
-                f"; sweep of {SAMPLE_ROWS} rows per linear at full width (scale n_out/{SAMPLE_ROWS}): "
-                + ", ".join(parts["sweep"]) + f"; {self.spent():.1f} s of CPU work timed")
+                "; sweep per distinct linear shape at full width (rows for 64 MB of running weights; scale "
+                "linears of the shape x n_out/rows): " + ", ".join(parts["sweep"]) +
+                f"; {self.spent():.1f} s of CPU work timed")
 
 
 def cpu_cores():
