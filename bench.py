@@ -52,6 +52,9 @@ def parse_args():
     p.add_argument("--e2e-steps", type=int, default=6)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--qlinear", action="store_true",
+                   help="measure the linear on the quantized checkpoint (decode, dequantization, GEMM) alone")
+    p.add_argument("--qlinear-shape", default="", help="with --qlinear: only the shapes whose name contains this")
     p.add_argument("--cpu-full-layer", action="store_true",
                    help="time the float64 oracle on the whole layer once (minutes of CPU) beside the sample estimate")
     return p.parse_args()
@@ -672,11 +675,92 @@ def run_cpu_full_layer(args):
             "s_per_layer_sample_estimate": round(est, 1), "estimate_over_measured": round(est / full, 3)}
 
 
+def run_qlinear(args):
+    """The linear on the quantized checkpoint (4-bit, group 128, act order), measured alone on
+    Llama-shaped weights quantized by the library itself: the decode kernel (M = 1 and 4 rows; HBM-bound: bytes =
+    packed codes + fp16 scales + packed zero points + g_idx + X + Y) against the measured
+    copy bandwidth, the dequantization (bytes = the checkpoint read + the 16-bit weight
+    written) likewise, and the tensor-core GEMM (2 M N K flops) against the measured bf16
+    rate.  CUDA events on the launching stream, 3 warm-ups, the median of 20 launches;
+    weights are re-read every launch (decode shapes below L2 are reported as such)."""
+    import torch
+
+    import post_weight_quantization_layer_b200 as gq
+    from post_weight_quantization_layer_b200 import synth
+    from post_weight_quantization_layer_b200._native import lib
+    peaks = load_peaks()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, reps=20):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    out = {"mode": "qlinear", "unit_decode": "GB/s", "unit_gemm": "TFLOP/s", "hbm_peak_gbs": peaks["hbm"],
+           "bf16_peak_tflops": peaks["bf16"], "peaks": peaks["source"], "shapes": []}
+    bits, g = 4, 128
+    shapes = (("7b q_proj", 4096, 4096), ("7b gate_proj", 4096, 11008), ("7b down_proj", 11008, 4096),
+              ("70b gate_proj", 8192, 28672), ("70b down_proj", 28672, 8192))
+    for name, n_in, n_out in shapes:
+        if args.qlinear_shape and args.qlinear_shape not in name:
+            continue
+        # a real checkpoint of the library's own making: Hessian, GPTQ with act order, export
+        W = synth.outlier_weight(n_out, n_in, 11, device=dev)
+        H = torch.zeros(n_in, n_in, device=dev)
+        acts = synth.StudentTActs(n_in, 2 * n_in, 12, dtype=torch.bfloat16)
+        for i in range(acts.n_chunks):
+            gq.accumulate_hessian(acts.get_chunk(i, device=dev), H)
+        res = gq.quantize_layer(W, H, bits, g, 0.01, True, True, False, 128)
+        del W, H
+        from post_weight_quantization_layer_b200.export import export_layer
+        ck = export_layer(res, bits)
+        G = ck["scales"].shape[0]
+        wbytes = n_in * n_out * bits // 8 + G * n_out * (2 + bits / 8) + n_in * 4
+        row = {"shape": name, "n_in": n_in, "n_out": n_out, "weight_bytes": int(wbytes)}
+        for M in (1, 4):
+            X = torch.randn(M, n_in, device=dev).to(torch.bfloat16)
+            Y = torch.empty(M, n_out, device=dev, dtype=torch.bfloat16)
+            ms = timed(lambda: gq.quantized_linear(X, ck, bits, out=Y))
+            gbs = (wbytes + M * (n_in + n_out) * 2) / (ms / 1e3) / 1e9
+            row[f"decode_m{M}"] = {"us": round(ms * 1e3, 1), "gbs": round(gbs, 1),
+                                   "frac_of_hbm": round(gbs / peaks["hbm"], 3),
+                                   "l2_resident": wbytes < 100e6}
+        Wd = torch.empty(n_out, n_in, dtype=torch.bfloat16, device=dev)
+        ms = timed(lambda: lib().gptq_dequantize_weight(ck["qweight"].data_ptr(), ck["qzeros"].data_ptr(),
+                                                         ck["scales"].data_ptr(), ck["g_idx"].data_ptr(), G, n_in,
+                                                         n_out, bits, 2, Wd.data_ptr(), stream.cuda_stream))
+        gbs = (wbytes + n_in * n_out * 2) / (ms / 1e3) / 1e9
+        row["dequant"] = {"us": round(ms * 1e3, 1), "gbs": round(gbs, 1), "frac_of_hbm": round(gbs / peaks["hbm"], 3)}
+        for M in (2048, 16384):
+            X = torch.randn(M, n_in, device=dev).to(torch.bfloat16)
+            Y = torch.empty(M, n_out, device=dev, dtype=torch.bfloat16)
+            ms = timed(lambda: gq.quantized_linear(X, ck, bits, out=Y), reps=10)
+            tf = 2 * M * n_in * n_out / (ms / 1e3) / 1e12
+            row[f"gemm_m{M}"] = {"ms": round(ms, 3), "tflops": round(tf, 1), "frac_of_bf16_burst": round(tf / peaks["bf16"], 3)}
+            del X, Y
+        out["shapes"].append(row)
+        del ck, Wd
+        torch.cuda.empty_cache()
+    return out
+
+
 def main():
     args = parse_args()
     world, rank, local = dist_setup(args.gpus)
     try:
-        if args.cpu_full_layer:
+        if args.qlinear:
+            line = run_qlinear(args) if rank == 0 else None
+        elif args.cpu_full_layer:
             line = run_cpu_full_layer(args) if rank == 0 else None
         elif args.impl == "reference":
             line = run_reference(args, world, rank)
