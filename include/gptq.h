@@ -124,8 +124,9 @@ int gptq_accumulate_hessian(const void* X, int x_dtype, int64_t tokens, int64_t 
  *   g_idx   [n_in] int32: group of each original input column.
  *   Dequantized weight: scales[g_idx[c], o] * (code[o, c] - zeros[g_idx[c], o]).
  * n_in*bits % 32 != 0 or n_in % 8 != 0 -> UNSUPPORTED.
- * Workspace (about 3*n_in^2*8 + n_out*n_in*17 bytes) is taken stream-ordered from a
- * library-owned pool that keeps it cached for later calls (OOM if that fails; see
+ * Workspace (about 3*n_in^2*8 + n_out*n_in*17 bytes, plus 10*(n_out + n_in)*B bytes of
+ * int8 operand slices for the lazy block updates, B = 256 or 512) is taken stream-ordered
+ * from a library-owned pool that keeps it cached for later calls (OOM if that fails; see
  * gptq_trim_workspace).  The call is blocking: it synchronises
  * `stream` once at the end and returns NOT_PD if a pivot failed.
  * stats may be NULL.

@@ -276,7 +276,8 @@ int gptq_test_wait_expiry(int skip_loads, uint32_t wait_limit) {
 int gptq_device_status(void* stream, int clear) {
   const int h = hessian_device_status(static_cast<cudaStream_t>(stream), clear);
   const int g = gemm_device_status(clear);
-  return h != GPTQ_OK ? h : g;
+  const int i = i8_device_status(clear);
+  return h != GPTQ_OK ? h : (g != GPTQ_OK ? g : i);
 }
 
 int gptq_factor_hessian(const float* H, int64_t n_in, float damp_percent, int desc_act, double* U, int32_t* perm,

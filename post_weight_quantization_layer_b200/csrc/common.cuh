@@ -89,6 +89,17 @@ int dgemm(cudaStream_t s, int64_t M, int64_t N, int64_t K, double alpha, const d
           const double* B, int64_t ldb, bool transB, double beta, double* C, int64_t ldc, bool upper,
           int tri = 0);
 
+// ozaki.cu: the sweep's trailing update C -= A B on the int8 tensor cores, A and B split
+// into signed 7-bit slices (rows of A, columns of B) with power-of-two scales.
+int i8_slices();
+int64_t i8_padded_k(int64_t K);
+int i8_split_rows(cudaStream_t s, const double* X, int64_t ldx, int64_t R, int64_t K, int64_t KP, int8_t* S, int* e);
+int i8_split_cols(cudaStream_t s, const double* Y, int64_t ldy, int64_t K, int64_t N, int64_t KP, int8_t* S, int* e);
+int i8_gemm_sub(cudaStream_t s, int64_t M, int64_t N, int64_t KP, const int8_t* SA, int64_t a_rows, const int* ea,
+                const int8_t* SB, int64_t b_cols, const int* eb, int64_t col0, double* C, int64_t ldc,
+                int max_ctas);
+int i8_device_status(int clear);
+
 // factor.cu: U (sweep order, fp64) and perm from H, stream-ordered on s.  `work` holds
 // factor_work_bytes(n, side != nullptr), `small` factor_small_bytes(n); `status` is a device
 // int.  With a side stream (and two events for its ordering) the top level's T product runs

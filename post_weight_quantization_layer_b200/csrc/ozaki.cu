@@ -1,0 +1,451 @@
+// The sweep's lazy trailing update on the 5th-generation int8 tensor cores.
+//
+// Source of the operation: "第5章 GPTQ 实战" §5.1.8 key point 3 (lazy batch update): after a
+// block of columns is quantized, its normalised errors update every later column at once,
+// W[:, later] -= Err[:, block] U[block, later].  The sweep needs this product to fp64-level
+// accuracy (its rounding decisions are chained), which the fp64 units give at ~37 TFLOP/s.
+// Here it is formed from exact integer products instead (a splitting of the operands into
+// small integer slices, as in Ozaki's scheme for accurate matrix products):
+//
+//   every row r of A = Err[:, block] is written A[r, k] ~ sum_{p<5} SA_p[r, k] 2^(ea_r - 7(p+1))
+//   every column n of B = U[block, later] is B[k, n] ~ sum_{q<5} SB_q[n, k] 2^(eb_n - 7(q+1))
+//   with SA_p, SB_q integers in [-127, 127] taken by repeated scaling by 2^7 and rounding to
+//   nearest (an unbiased remainder: truncation's bias accumulated over the sweep's blocks and
+//   flipped near-tie codes), and 2^ea_r > max |A[r, :]|, 2^eb_n > max |B[:, n]|.  Then
+//   (A B)[r, n] ~ 2^(ea_r + eb_n) sum_{s<5} 2^(-7(s+2)) sum_{p+q=s} (SA_p SB_q^T)[r, n],
+//   keeping the 15 slice pairs with p + q <= 4 (35 bits of each operand; four slices, 28
+//   bits, left a few more near-tie flips than fp64 in the parity tests).  Each SA_p SB_q^T
+//   is an exact int32 product (127^2 * K * 5 < 2^31 for K <= 16384).
+//
+// Kernels: split_rows_kernel / split_cols_kernel write the slices K-major (k contiguous)
+// for TMA; i8_gemm_kernel runs tcgen05.mma kind::i8 (s8 x s8 -> s32) with the U slices as
+// the M side (128 later columns) and the Err slices as the N side (48 rows of W), five TMEM
+// accumulators (one per s = p + q), double buffered, a 2-stage TMA ring of all slices of a
+// 64-wide K step (64-byte swizzle).  Its 111 KB of shared memory and 160 registers a thread
+// leave room on the SM for one CTA of the sweep's panel kernel, which runs beside it.  In
+// the epilogue a thread owns one column and a warp updates 32 consecutive columns of a row
+// at a time (coalesced fp64 read-modify-write, loads issued together); each element of W is
+// updated by exactly one thread of one CTA per launch (deterministic).
+#include <cuda.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace gptq {
+namespace {
+
+using namespace sm100;
+
+constexpr int KS = 5;        // slices per operand
+constexpr int SBETA = 7;     // bits per slice
+constexpr int IBM = 128;     // later columns of W per tile (UMMA M: the U slices)
+constexpr int IBN = 48;      // rows of W per tile (UMMA N: the Err slices)
+constexpr int IBK = 64;      // K (bytes = int8 elements) per stage: one 64-byte swizzle row
+constexpr int ISTAGES = 2;
+constexpr int IA_BYTES = KS * IBM * IBK;  // 40 KiB: U slices (UMMA A)
+constexpr int IB_BYTES = KS * IBN * IBK;  // 15 KiB: Err slices (UMMA B)
+constexpr int ISTAGE_BYTES = IA_BYTES + IB_BYTES;
+constexpr int ITHREADS = 320;
+constexpr int ISMEM = ISTAGES * ISTAGE_BYTES + 1024 + 256;
+constexpr uint32_t IWAIT = 1u << 24;
+
+__device__ int g_i8_status = 0;
+
+// ------------------------------------------------------------------ splitting
+// One warp per row of A (rows of Err[:, block], K = block width): the row exponent, then
+// KS slices of every element.  S is [KS][R][KP] (k contiguous, zero padded to KP).
+__global__ void split_rows_kernel(const double* __restrict__ X, int64_t ldx, int64_t R, int64_t K, int64_t KP,
+                                  int8_t* __restrict__ S, int* __restrict__ e) {
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (r >= R) return;
+  double m = 0.0;
+  for (int64_t k = lane; k < K; k += 32) m = fmax(m, fabs(X[r * ldx + k]));
+  for (int off = 16; off; off >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, off));
+  const int ex = m > 0.0 ? ilogb(m) + 1 : 0;  // 2^ex > m
+  if (lane == 0) e[r] = ex;
+  for (int64_t k = lane; k < KP; k += 32) {
+    double v = k < K ? ldexp(X[r * ldx + k], -ex) : 0.0;  // |v| < 1
+#pragma unroll
+    for (int p = 0; p < KS; ++p) {
+      v *= 128.0;
+      const double sl = fmin(fmax(rint(v), -127.0), 127.0);  // nearest, |v - sl| <= 1
+      v -= sl;
+      S[(static_cast<int64_t>(p) * R + r) * KP + k] = static_cast<int8_t>(sl);
+    }
+  }
+}
+
+// Columns of B = U[block, later] (row-major, ldy): 32 columns per CTA, the column exponent,
+// then the slices transposed through shared memory into S [KS][N][KP] (k contiguous).
+__global__ void __launch_bounds__(256) split_cols_kernel(const double* __restrict__ Y, int64_t ldy, int64_t K,
+                                                         int64_t N, int64_t KP, int8_t* __restrict__ S,
+                                                         int* __restrict__ e) {
+  __shared__ double mx[8][32];
+  __shared__ int exs[32];
+  __shared__ int8_t tile[KS][32][33];
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int64_t n = static_cast<int64_t>(blockIdx.x) * 32 + tx;
+  double m = 0.0;
+  if (n < N)
+    for (int64_t k = ty; k < K; k += 8) m = fmax(m, fabs(Y[k * ldy + n]));
+  mx[ty][tx] = m;
+  __syncthreads();
+  if (ty == 0) {
+    double mm = 0.0;
+    for (int i = 0; i < 8; ++i) mm = fmax(mm, mx[i][tx]);
+    const int ex = mm > 0.0 ? ilogb(mm) + 1 : 0;
+    exs[tx] = ex;
+    if (n < N) e[n] = ex;
+  }
+  __syncthreads();
+  for (int64_t k0 = 0; k0 < KP; k0 += 32) {
+    for (int kk = ty; kk < 32; kk += 8) {
+      const int64_t k = k0 + kk;
+      double v = (n < N && k < K) ? ldexp(Y[k * ldy + n], -exs[tx]) : 0.0;
+#pragma unroll
+      for (int p = 0; p < KS; ++p) {
+        v *= 128.0;
+        const double sl = fmin(fmax(rint(v), -127.0), 127.0);
+        v -= sl;
+        tile[p][tx][kk] = static_cast<int8_t>(sl);
+      }
+    }
+    __syncthreads();
+    for (int cc = ty; cc < 32; cc += 8) {
+      const int64_t nn = static_cast<int64_t>(blockIdx.x) * 32 + cc;
+      if (nn < N)
+        for (int p = 0; p < KS; ++p) S[(static_cast<int64_t>(p) * N + nn) * KP + k0 + tx] = tile[p][cc][tx];
+    }
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------------ tcgen05 kind::i8 GEMM
+// 32 lanes x 16 consecutive 32-bit columns, the wait in the same statement.
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, int (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+// Shared-memory descriptor, K-major with 64-byte swizzle: rows of 64 bytes, 8-row atoms of 512
+// bytes (stride-dimension offset); the leading-dimension offset is unused (one MMA's K, 32
+// bytes, lies inside a swizzle row).
+__device__ __forceinline__ uint64_t desc_sw64(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(1u) << 16;
+  d |= static_cast<uint64_t>((512u >> 4) & 0x3FFFu) << 32;
+  d |= 1ull << 46;
+  d |= 4ull << 61;
+  return d;
+}
+
+__device__ __forceinline__ void umma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Instruction descriptor of kind::i8: D s32 (2), A and B signed 8-bit (1), both K-major.
+__host__ __device__ constexpr uint32_t i8_idesc(int M, int N) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | ((static_cast<uint32_t>(N) >> 3) << 17) |
+         ((static_cast<uint32_t>(M) >> 4) << 24);
+}
+
+struct I8Args {
+  int M, N, KP;               // rows, columns, padded K
+  int a_rows, b_cols;         // slice strides (rows of SA per slice, columns of SB per slice)
+  const int* ea;              // [a_rows] row exponents
+  const int* eb;              // [b_cols] column exponents (for columns col0 ...)
+  int col0;                   // first column of this launch within SB / eb
+  double* C;                  // C[r, c] for c in [0, N): C + r * ldc + c
+  int64_t ldc;
+  int mt, nt;
+};
+
+__global__ void __maxnreg__(160)
+    i8_gemm_kernel(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb, I8Args a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + ISTAGES * ISTAGE_BYTES);
+  uint64_t* empty = full + ISTAGES;
+  uint64_t* accf = empty + ISTAGES;
+  uint64_t* acce = accf + 2;
+  uint64_t* done = acce + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = static_cast<int>(gridDim.x);
+  const int units = a.mt * a.nt;
+  const int nk = a.KP / IBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < ISTAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accf[b], 1);
+      mbar_init(&acce[b], 8);
+    }
+    mbar_init(done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  bool ok = true;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer: all KS slices of A and B for one 128-wide K step
+      tma_prefetch_desc(&ta);
+      tma_prefetch_desc(&tb);
+      int stage = 0, issued = 0;
+      uint32_t ph = 0;
+      for (int u = blockIdx.x; u < units && ok; u += G) {
+        const int c0 = a.col0 + (u / a.mt) * IBM, r0 = (u % a.mt) * IBN;
+        for (int ks = 0; ks < nk; ++ks) {
+          if (!mbar_wait(&empty[stage], ph ^ 1u, IWAIT)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * ISTAGE_BYTES;
+          uint8_t* sb = sa + IA_BYTES;
+          mbar_arrive_expect_tx(&full[stage], ISTAGE_BYTES);
+#pragma unroll
+          for (int p = 0; p < KS; ++p) {
+            tma_load_2d(sa + p * IBM * IBK, &tb, &full[stage], ks * IBK, p * a.b_cols + c0);
+            tma_load_2d(sb + p * IBN * IBK, &ta, &full[stage], ks * IBK, p * a.a_rows + r0);
+          }
+          ++issued;
+          if (++stage == ISTAGES) {
+            stage = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      for (int k = 0; k < min(issued, ISTAGES); ++k) {
+        int s = stage - 1 - k;
+        uint32_t p = ph;
+        while (s < 0) {
+          s += ISTAGES;
+          p ^= 1u;
+        }
+        mbar_wait(&full[s], p, IWAIT);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- UMMA issuer: 15 slice pairs (p + q <= 4) per 32-wide K substep
+      constexpr uint32_t idesc = i8_idesc(IBM, IBN);
+      int stage = 0, cg = 0;
+      uint32_t ph = 0;
+      for (int u = blockIdx.x; u < units && ok; u += G, ++cg) {
+        const int b = cg & 1;
+        if (!mbar_wait(&acce[b], ((cg >> 1) & 1) ^ 1u, IWAIT)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t dbase = tmem + static_cast<uint32_t>(b * KS * IBN);
+        for (int ks = 0; ks < nk; ++ks) {
+          if (!mbar_wait(&full[stage], ph, IWAIT)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * ISTAGE_BYTES);
+          const uint32_t sb = sa + IA_BYTES;
+#pragma unroll
+          for (int k = 0; k < IBK / 32; ++k) {
+#pragma unroll
+            for (int p = 0; p < KS; ++p)
+#pragma unroll
+              for (int q = 0; q < KS - p; ++q) {
+                const uint64_t ad = desc_sw64(sa + p * IBM * IBK + k * 32);
+                const uint64_t bd = desc_sw64(sb + q * IBN * IBK + k * 32);
+                // pairs go p-major, so (0, s) is the first product into accumulator s: it
+                // overwrites the accumulator's previous tile
+                const bool first = ks == 0 && k == 0 && p == 0;
+                umma_i8(dbase + static_cast<uint32_t>((p + q) * IBN), ad, bd, idesc, first ? 0u : 1u);
+              }
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == ISTAGES) {
+            stage = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&accf[b]);
+      }
+      umma_commit(done);
+      mbar_wait(done, 0, IWAIT);
+    }
+  } else {
+    // ---------------- epilogue: C[r, n] -= 2^(ea_r + eb_n - 14) sum_s acc_s 2^(-7 s).  A thread
+    // owns one column n (its TMEM lane); the 4 warps of each lane quarter are split over the
+    // tile's 48 rows in chunks of 16 (warps 2..5 and 6..9 take chunks 0, 2 and 1); for each
+    // row the warp's 32 lanes update 32 consecutive columns (coalesced).  The 16 loads of W are
+    // issued together before any use.
+    const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
+    int cg = 0;
+    for (int u = blockIdx.x; u < units; u += G, ++cg) {
+      const int b = cg & 1;
+      if (!mbar_wait(&accf[b], (cg >> 1) & 1, IWAIT)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int c = (u / a.mt) * IBM + quad * 32 + lane;  // column within this launch
+      const bool cin = c < a.N;
+      const int ec = cin ? a.eb[a.col0 + c] - 2 * SBETA : 0;
+      for (int chunk = half; chunk < IBN / 16; chunk += 2) {
+        const int r0 = (u % a.mt) * IBN + chunk * 16;
+        int acc[KS][16];
+#pragma unroll
+        for (int s = 0; s < KS; ++s)
+          tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(quad * 32) << 16) +
+                                 static_cast<uint32_t>(b * KS * IBN + s * IBN + chunk * 16),
+                             acc[s]);
+        double cv[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          cv[j] = (cin && r0 + j < a.M) ? a.C[static_cast<int64_t>(r0 + j) * a.ldc + c] : 0.0;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          double v = static_cast<double>(acc[KS - 1][j]);
+#pragma unroll
+          for (int s = KS - 2; s >= 0; --s) v = fma(v, 0x1p-7, static_cast<double>(acc[s][j]));
+          if (cin && r0 + j < a.M) a.C[static_cast<int64_t>(r0 + j) * a.ldc + c] = cv[j] - ldexp(v, ec + a.ea[r0 + j]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acce[b]);  // this warp's reads of the accumulators are done
+    }
+  }
+  if (!ok) atomicExch(&g_i8_status, kStatusTimeout);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<EncodeTiledFn>(p);
+    return static_cast<EncodeTiledFn>(nullptr);
+  }();
+  return fn;
+}
+
+// rows x KP int8, boxes of 64 (K) x box_rows, 64-byte swizzle
+int slice_map(CUtensorMap* tm, const int8_t* base, int64_t rows, int64_t KP, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return GPTQ_ERR_CUDA;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(KP), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(KP)};
+  cuuint32_t box[2] = {IBK, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? GPTQ_OK : GPTQ_ERR_CUDA;
+}
+
+}  // namespace
+
+int i8_slices() { return KS; }
+int64_t i8_padded_k(int64_t K) { return ((K + IBK - 1) / IBK) * IBK; }
+
+int i8_split_rows(cudaStream_t s, const double* X, int64_t ldx, int64_t R, int64_t K, int64_t KP, int8_t* S, int* e) {
+  if (R <= 0) return GPTQ_OK;
+  split_rows_kernel<<<static_cast<unsigned>((R + 7) / 8), 256, 0, s>>>(X, ldx, R, K, KP, S, e);
+  return after_launch();
+}
+
+int i8_split_cols(cudaStream_t s, const double* Y, int64_t ldy, int64_t K, int64_t N, int64_t KP, int8_t* S, int* e) {
+  if (N <= 0) return GPTQ_OK;
+  split_cols_kernel<<<static_cast<unsigned>((N + 31) / 32), 256, 0, s>>>(Y, ldy, K, N, KP, S, e);
+  return after_launch();
+}
+
+// C[r, c] -= (A B)[r, col0 + c] for r < M, c < N, from the slices of i8_split_rows (SA,
+// a_rows rows per slice, exponents ea) and i8_split_cols (SB, b_cols columns per slice,
+// exponents eb), K padded to KP.  The persistent grid has at most max_ctas CTAs (0: one per
+// SM): a CTA takes most of an SM's shared memory, so a launch that runs beside other
+// kernels leaves them SMs of their own.
+int i8_gemm_sub(cudaStream_t s, int64_t M, int64_t N, int64_t KP, const int8_t* SA, int64_t a_rows, const int* ea,
+                const int8_t* SB, int64_t b_cols, const int* eb, int64_t col0, double* C, int64_t ldc,
+                int max_ctas) {
+  if (M <= 0 || N <= 0) return GPTQ_OK;
+  // Rows past a slice's end (a tile reaching beyond M) load the next slice's first rows, or
+  // zeros past the last slice; they only reach accumulator rows (columns) >= M (N), which
+  // the epilogue never writes.
+  if (KP % IBK != 0 || KP > 16384 || M > a_rows || col0 + N > b_cols) return GPTQ_ERR_UNSUPPORTED;
+  GPTQ_TRY(ensure_smem_limit(reinterpret_cast<const void*>(i8_gemm_kernel), ISMEM));
+  CUtensorMap ta, tb;
+  GPTQ_TRY(slice_map(&ta, SA, KS * a_rows, KP, IBN));
+  GPTQ_TRY(slice_map(&tb, SB, KS * b_cols, KP, IBM));
+  I8Args a;
+  a.M = static_cast<int>(M);
+  a.N = static_cast<int>(N);
+  a.KP = static_cast<int>(KP);
+  a.a_rows = static_cast<int>(a_rows);
+  a.b_cols = static_cast<int>(b_cols);
+  a.ea = ea;
+  a.eb = eb;
+  a.col0 = static_cast<int>(col0);
+  a.C = C;
+  a.ldc = ldc;
+  a.mt = static_cast<int>((M + IBN - 1) / IBN);  // row tiles of 64
+  a.nt = static_cast<int>((N + IBM - 1) / IBM);  // column tiles of 128
+  const int cap = max_ctas > 0 ? std::min(max_ctas, num_sms()) : num_sms();
+  const int grid = static_cast<int>(std::min<int64_t>(cap, static_cast<int64_t>(a.mt) * a.nt));
+  i8_gemm_kernel<<<grid, ITHREADS, ISMEM, s>>>(ta, tb, a);
+  return after_launch();
+}
+
+int i8_device_status(int clear) {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_i8_status, sizeof(int)) != cudaSuccess) return GPTQ_ERR_CUDA;
+  if (clear) {
+    int z = 0;
+    if (cudaMemcpyToSymbol(g_i8_status, &z, sizeof(int)) != cudaSuccess) return GPTQ_ERR_CUDA;
+  }
+  return v;
+}
+
+}  // namespace gptq

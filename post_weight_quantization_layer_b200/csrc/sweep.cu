@@ -25,14 +25,13 @@
 // * Two-level lazy updates: inside an outer block (<= 512 columns) each panel kernel first
 //   applies the pending errors of the block's earlier panels to its own columns (a small
 //   left-looking product on the fp64 matrix units); after each outer block its errors
-//   update every later column in one GEMM with K = outer block width.
-// * Look-ahead: that GEMM is split in two.  The next outer block's columns are updated
-//   first, on a high-priority stream that then runs the next block's panels; the rest of
-//   the trailing update runs at the same time on a low-priority stream.  The panel chain
-//   (latency-bound, one CTA of 4 warps per SM) shares the SMs with the GEMM's tiles
-//   (one CTA per SM), so the two overlap; where a panel shares its SM with a GEMM CTA its
-//   fp64 instructions wait behind the GEMM's on the shared fp64 pipe, and the panel
-//   chain remains the longer of the two.
+//   update every later column at once.  That trailing update runs on the int8 tensor cores
+//   (ozaki.cu: both operands split into five 7-bit slices, exact integer slice products,
+//   fp64 recombination), which leaves the fp64 pipe to the panels' compensation chain.
+// * Look-ahead: the trailing update is split in two.  The next outer block's columns are
+//   updated first, on a high-priority stream that then runs the next block's panels; the
+//   rest runs at the same time on a low-priority stream.  A panel CTA and a trailing-update
+//   CTA fit on one SM together (shared memory and registers), so the two overlap.
 #include <algorithm>
 
 #include "common.cuh"
@@ -567,6 +566,39 @@ int run_sweep(SweepArgs& a, cudaStream_t s, int* panel_width, int* outer_width) 
   pa.loss = a.loss;
   const unsigned panel_grid = static_cast<unsigned>((n_out + ROWS - 1) / ROWS);
 
+  // Slices of the trailing update's operands (int8 tensor cores): two sets, by outer-block
+  // parity.  Block b+1 splits into the set that block b-1 used; block b-1's last reader of
+  // it, its trailing GEMM on the low-priority lane, finished before block b's look-ahead
+  // (which waits for it) and so before block b+1's panels and split on the panel lane.
+  const int64_t KP = i8_padded_k(Q);
+  const bool use_i8 = KP <= 16384;
+  const int KSL = i8_slices();
+  int8_t* SA[2] = {nullptr, nullptr};
+  int8_t* SB[2] = {nullptr, nullptr};
+  int* EA[2] = {nullptr, nullptr};
+  int* EB[2] = {nullptr, nullptr};
+  void* slices = nullptr;
+  if (use_i8 && Q < n_in) {
+    const size_t sa = (static_cast<size_t>(KSL) * n_out * KP + 255) & ~size_t(255);
+    const size_t sb = (static_cast<size_t>(KSL) * n_in * KP + 255) & ~size_t(255);
+    const size_t ea = (static_cast<size_t>(n_out) * 4 + 255) & ~size_t(255);
+    const size_t eb = (static_cast<size_t>(n_in) * 4 + 255) & ~size_t(255);
+    GPTQ_TRY(pool_alloc(&slices, 2 * (sa + sb + ea + eb), s));
+    char* p = static_cast<char*>(slices);
+    for (int b = 0; b < 2; ++b) {
+      SA[b] = reinterpret_cast<int8_t*>(p);
+      SB[b] = reinterpret_cast<int8_t*>(p + sa);
+      EA[b] = reinterpret_cast<int*>(p + sa + sb);
+      EB[b] = reinterpret_cast<int*>(p + sa + sb + ea);
+      p += sa + sb + ea + eb;
+    }
+  }
+  struct FreeOnExit {
+    void* p;
+    cudaStream_t s;
+    ~FreeOnExit() { pool_free(p, s); }
+  } free_slices{slices, s};  // declared before the lanes: freed after they join into s
+
   {
     LaneLease lanes(s);
     const LanePrio prio[2] = {kLaneHigh, kLaneLow};  // panels + look-ahead; trailing update
@@ -593,17 +625,31 @@ int run_sweep(SweepArgs& a, cudaStream_t s, int* panel_width, int* outer_width) 
       }
       if (O1 >= n_in) break;
       // Err[:, O0:O1] is complete: every later column gets W -= Err[:, O0:O1] U[O0:O1, :].
+      const int bp = static_cast<int>((O0 / Q) & 1);
+      const int64_t nl = n_in - O1;  // later columns
+      if (use_i8) {
+        GPTQ_TRY(i8_split_rows(sp, a.Err + O0, n_in, n_out, O1 - O0, KP, SA[bp], EA[bp]));
+        GPTQ_TRY(i8_split_cols(sp, a.U + O0 * n_in + O1, n_in, O1 - O0, nl, KP, SB[bp], EB[bp]));
+      }
       GPTQ_CUDA(cudaEventRecord(pan, sp));
       // The next block's columns first (on the panel stream, so its panels follow at once);
       // they were last written by the previous block's trailing update.
       if (rest_issued) GPTQ_CUDA(cudaStreamWaitEvent(sp, rest, 0));
-      GPTQ_TRY(dgemm(sp, n_out, O2 - O1, O1 - O0, -1.0, a.Err + O0, n_in, a.U + O0 * n_in + O1, n_in, false, 1.0,
-                     a.Wk + O1, n_in, false));
+      if (use_i8)
+        GPTQ_TRY(i8_gemm_sub(sp, n_out, O2 - O1, KP, SA[bp], n_out, EA[bp], SB[bp], nl, EB[bp], 0, a.Wk + O1, n_in,
+                             0));
+      else
+        GPTQ_TRY(dgemm(sp, n_out, O2 - O1, O1 - O0, -1.0, a.Err + O0, n_in, a.U + O0 * n_in + O1, n_in, false, 1.0,
+                       a.Wk + O1, n_in, false));
       // Every column after the next block, concurrently with the next block's panels.
       if (O2 < n_in) {
         GPTQ_CUDA(cudaStreamWaitEvent(sg, pan, 0));
-        GPTQ_TRY(dgemm(sg, n_out, n_in - O2, O1 - O0, -1.0, a.Err + O0, n_in, a.U + O0 * n_in + O2, n_in, false,
-                       1.0, a.Wk + O2, n_in, false));
+        if (use_i8)
+          GPTQ_TRY(i8_gemm_sub(sg, n_out, n_in - O2, KP, SA[bp], n_out, EA[bp], SB[bp], nl, EB[bp], O2 - O1,
+                               a.Wk + O2, n_in, 0));
+        else
+          GPTQ_TRY(dgemm(sg, n_out, n_in - O2, O1 - O0, -1.0, a.Err + O0, n_in, a.U + O0 * n_in + O2, n_in, false,
+                         1.0, a.Wk + O2, n_in, false));
         GPTQ_CUDA(cudaEventRecord(rest, sg));
         rest_issued = true;
       }
