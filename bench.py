@@ -676,8 +676,8 @@ def run_cpu_full_layer(args):
 
 
 def run_qlinear(args):
-    """The linear on the quantized checkpoint (4-bit, group 128, act order), measured alone on
-    Llama-shaped weights quantized by the library itself: the decode kernel (M = 1 and 4 rows; HBM-bound: bytes =
+    """The linear on the quantized checkpoint (4-bit, group 128; act order, and for decoding also
+    without it), measured alone on Llama-shaped weights quantized by the library itself: the decode kernel (M = 1 and 4 rows; HBM-bound: bytes =
     packed codes + fp16 scales + packed zero points + g_idx + X + Y) against the measured
     copy bandwidth, the dequantization (bytes = the checkpoint read + the 16-bit weight
     written) likewise, and the tensor-core GEMM (2 M N K flops) against the measured bf16
@@ -720,21 +720,22 @@ def run_qlinear(args):
         acts = synth.StudentTActs(n_in, 2 * n_in, 12, dtype=torch.bfloat16)
         for i in range(acts.n_chunks):
             gq.accumulate_hessian(acts.get_chunk(i, device=dev), H)
-        res = gq.quantize_layer(W, H, bits, g, 0.01, True, True, False, 128)
-        del W, H
         from post_weight_quantization_layer_b200.export import export_layer
-        ck = export_layer(res, bits)
+        ck = export_layer(gq.quantize_layer(W, H, bits, g, 0.01, True, True, False, 128), bits)
+        ck_mono = export_layer(gq.quantize_layer(W, H, bits, g, 0.01, True, False, False, 128), bits)
+        del W, H
         G = ck["scales"].shape[0]
         wbytes = n_in * n_out * bits // 8 + G * n_out * (2 + bits / 8) + n_in * 4
         row = {"shape": name, "n_in": n_in, "n_out": n_out, "weight_bytes": int(wbytes)}
-        for M in (1, 4):
-            X = torch.randn(M, n_in, device=dev).to(torch.bfloat16)
-            Y = torch.empty(M, n_out, device=dev, dtype=torch.bfloat16)
-            ms = timed(lambda: gq.quantized_linear(X, ck, bits, out=Y))
-            gbs = (wbytes + M * (n_in + n_out) * 2) / (ms / 1e3) / 1e9
-            row[f"decode_m{M}"] = {"us": round(ms * 1e3, 1), "gbs": round(gbs, 1),
-                                   "frac_of_hbm": round(gbs / peaks["hbm"], 3),
-                                   "l2_resident": wbytes < 100e6}
+        for tag, c in (("", ck), ("_monotone_groups", ck_mono)):
+            for M in (1, 4):
+                X = torch.randn(M, n_in, device=dev).to(torch.bfloat16)
+                Y = torch.empty(M, n_out, device=dev, dtype=torch.bfloat16)
+                ms = timed(lambda: gq.quantized_linear(X, c, bits, out=Y))
+                gbs = (wbytes + M * (n_in + n_out) * 2) / (ms / 1e3) / 1e9
+                row[f"decode_m{M}{tag}"] = {"us": round(ms * 1e3, 1), "gbs": round(gbs, 1),
+                                            "frac_of_hbm": round(gbs / peaks["hbm"], 3),
+                                            "l2_resident": wbytes < 100e6}
         Wd = torch.empty(n_out, n_in, dtype=torch.bfloat16, device=dev)
         ms = timed(lambda: lib().gptq_dequantize_weight(ck["qweight"].data_ptr(), ck["qzeros"].data_ptr(),
                                                          ck["scales"].data_ptr(), ck["g_idx"].data_ptr(), G, n_in,

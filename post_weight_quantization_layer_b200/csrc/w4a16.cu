@@ -113,6 +113,20 @@ constexpr uint32_t GWAIT = 1u << 24;
 
 __device__ int g_gemm_status = 0;
 
+// Tile order: bands of GM row tiles; inside a band the row tile varies fastest, so a wave of
+// CTAs covers GM row tiles x (wave / GM) column tiles and both operands' tiles of the wave
+// stay in L2 (a band of X and a slice of the weight), instead of each wave streaming the
+// whole weight for one row tile.
+constexpr int GM_BAND = 16;
+__device__ __forceinline__ void gemm_tile_at(int u, int mt, int nt, int& m_tile, int& n_tile) {
+  const int band = u / (GM_BAND * nt);
+  const int m_first = band * GM_BAND;
+  const int bm = min(GM_BAND, mt - m_first);
+  const int rem = u - band * GM_BAND * nt;
+  n_tile = rem / bm;
+  m_tile = m_first + rem % bm;
+}
+
 // K-major operand, 128-byte swizzle: rows of 64 16-bit elements (128 bytes), 8-row atoms of
 // 1024 bytes (stride-dimension offset); the leading-dimension offset is unused because one
 // MMA's K (16 elements, 32 bytes) lies inside a swizzle row.  K steps inside the row
@@ -167,7 +181,9 @@ __global__ void __launch_bounds__(GTHREADS, 1)
       int stage = 0, issued = 0;
       uint32_t ph = 0;
       for (int u = blockIdx.x; u < units && ok; u += G) {
-        const int m0 = (u / nt) * GBM, n0 = (u % nt) * GBN;
+        int mi, ni;
+        gemm_tile_at(u, mt, nt, mi, ni);
+        const int m0 = mi * GBM, n0 = ni * GBN;
         for (int ks = 0; ks < nk; ++ks) {
           if (!mbar_wait(&empty[stage], ph ^ 1u, GWAIT)) {
             ok = false;
@@ -244,8 +260,10 @@ __global__ void __launch_bounds__(GTHREADS, 1)
         break;
       }
       tc_fence_after();
-      const int m = (u / nt) * GBM + quad * 32 + lane;
-      const int nb = (u % nt) * GBN + half * 128;
+      int mi, ni;
+      gemm_tile_at(u, mt, nt, mi, ni);
+      const int m = mi * GBM + quad * 32 + lane;
+      const int nb = ni * GBN + half * 128;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         float v[32];
@@ -285,7 +303,7 @@ constexpr int GV_THREADS = 256;  // 8 warps; a lane owns 4 consecutive outputs
 constexpr int GV_N = 128;        // outputs per CTA
 constexpr int GV_MAXM = 4;
 
-template <int BITS, typename T>
+template <int BITS, typename T, int MM>
 __global__ void __launch_bounds__(GV_THREADS) gemv_kernel(const T* __restrict__ X, int M, int64_t K,
                                                           const int32_t* __restrict__ qweight,
                                                           const int32_t* __restrict__ qzeros,
@@ -304,13 +322,13 @@ __global__ void __launch_bounds__(GV_THREADS) gemv_kernel(const T* __restrict__ 
   for (int e = tid; e < kn; e += GV_THREADS) {
     gs[e] = clamp_group(__ldg(g_idx + klo + e), G);
 #pragma unroll
-    for (int m = 0; m < GV_MAXM; ++m) xs[m * kchunk + e] = m < M ? to_f32<T>(X[m * K + klo + e]) : 0.f;
+    for (int m = 0; m < MM; ++m) xs[m * kchunk + e] = to_f32<T>(X[m * K + klo + e]);
   }
   __syncthreads();
   const int64_t n = static_cast<int64_t>(blockIdx.x) * GV_N + lane * 4;
-  float acc[GV_MAXM][4];
+  float acc[MM][4];
 #pragma unroll
-  for (int m = 0; m < GV_MAXM; ++m)
+  for (int m = 0; m < MM; ++m)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[m][j] = 0.f;
   if (n < N) {
@@ -320,9 +338,8 @@ __global__ void __launch_bounds__(GV_THREADS) gemv_kernel(const T* __restrict__ 
     int gcur = -1;
     float s[4];
     int z[4];
-    for (int r = warp; r < rows; r += 8) {
-      const int64_t wrow = klo / FPW + r;
-      const int4 w4 = __ldg(reinterpret_cast<const int4*>(qweight + wrow * N + n));
+    // one word row of 4 outputs: its FPW codes each, with the group parameters of each code's k
+    auto row_math = [&](int r, const int4 w4) {
       const uint32_t wv[4] = {static_cast<uint32_t>(w4.x), static_cast<uint32_t>(w4.y), static_cast<uint32_t>(w4.z),
                               static_cast<uint32_t>(w4.w)};
 #pragma unroll
@@ -346,18 +363,27 @@ __global__ void __launch_bounds__(GV_THREADS) gemv_kernel(const T* __restrict__ 
         for (int j = 0; j < 4; ++j) {
           const float w = dq<T>(s[j], static_cast<int>((wv[j] >> (f * BITS)) & MASK), z[j]);
 #pragma unroll
-          for (int m = 0; m < GV_MAXM; ++m) acc[m][j] = fmaf(xs[m * kchunk + kl], w, acc[m][j]);
+          for (int m = 0; m < MM; ++m) acc[m][j] = fmaf(xs[m * kchunk + kl], w, acc[m][j]);
         }
       }
+    };
+    const int64_t wbase = klo / FPW;
+    int r = warp;
+    for (; r + 8 < rows; r += 16) {  // two word rows in flight
+      const int4 wa = __ldg(reinterpret_cast<const int4*>(qweight + (wbase + r) * N + n));
+      const int4 wb = __ldg(reinterpret_cast<const int4*>(qweight + (wbase + r + 8) * N + n));
+      row_math(r, wa);
+      row_math(r + 8, wb);
     }
+    if (r < rows) row_math(r, __ldg(reinterpret_cast<const int4*>(qweight + (wbase + r) * N + n)));
   }
   // the 8 warps' partial sums of this CTA's outputs, added in a fixed order
 #pragma unroll
-  for (int m = 0; m < GV_MAXM; ++m)
+  for (int m = 0; m < MM; ++m)
 #pragma unroll
     for (int j = 0; j < 4; ++j) red[(warp * GV_MAXM + m) * GV_N + lane * 4 + j] = acc[m][j];
   __syncthreads();
-  for (int e = tid; e < GV_MAXM * GV_N; e += GV_THREADS) {
+  for (int e = tid; e < MM * GV_N; e += GV_THREADS) {
     const int m = e / GV_N, c = e % GV_N;
     const int64_t nn = static_cast<int64_t>(blockIdx.x) * GV_N + c;
     if (m < M && nn < N) {
@@ -441,7 +467,7 @@ int dequant_any(int bits, const int32_t* qw, const int32_t* qz, const __half* sc
   return launch_dequant<8, T>(qw, qz, sc, gi, G, K, N, W, s);
 }
 
-template <int BITS, typename T>
+template <int BITS, typename T, int MM>
 int launch_gemv(const T* X, int M, int64_t K, const int32_t* qw, const int32_t* qz, const __half* sc,
                 const int32_t* gi, int G, int64_t N, T* Y, cudaStream_t s) {
   // K split so that about four CTAs per SM stream the weights; every split a multiple of
@@ -453,10 +479,10 @@ int launch_gemv(const T* X, int M, int64_t K, const int32_t* qw, const int32_t* 
   S = (K + kchunk - 1) / kchunk;
   if (S > 65535) return GPTQ_ERR_UNSUPPORTED;
   const size_t smem = (GV_MAXM * kchunk + kchunk) * 4 + 8 * GV_MAXM * GV_N * 4;
-  GPTQ_TRY(ensure_smem_limit(reinterpret_cast<const void*>(gemv_kernel<BITS, T>), static_cast<int>(smem)));
+  GPTQ_TRY(ensure_smem_limit(reinterpret_cast<const void*>(gemv_kernel<BITS, T, MM>), static_cast<int>(smem)));
   float* partial = nullptr;
   GPTQ_TRY(pool_alloc(reinterpret_cast<void**>(&partial), static_cast<size_t>(S) * M * N * 4, s));
-  gemv_kernel<BITS, T><<<dim3(static_cast<unsigned>(nblk), static_cast<unsigned>(S)), GV_THREADS, smem, s>>>(
+  gemv_kernel<BITS, T, MM><<<dim3(static_cast<unsigned>(nblk), static_cast<unsigned>(S)), GV_THREADS, smem, s>>>(
       X, M, K, qw, qz, sc, gi, G, N, static_cast<int>(kchunk), partial);
   int st = after_launch();
   if (st == GPTQ_OK) {
@@ -468,12 +494,23 @@ int launch_gemv(const T* X, int M, int64_t K, const int32_t* qw, const int32_t* 
   return st;
 }
 
+template <int BITS, typename T>
+int gemv_rows(const T* X, int M, int64_t K, const int32_t* qw, const int32_t* qz, const __half* sc,
+              const int32_t* gi, int G, int64_t N, T* Y, cudaStream_t s) {
+  switch (M) {
+    case 1: return launch_gemv<BITS, T, 1>(X, M, K, qw, qz, sc, gi, G, N, Y, s);
+    case 2: return launch_gemv<BITS, T, 2>(X, M, K, qw, qz, sc, gi, G, N, Y, s);
+    case 3: return launch_gemv<BITS, T, 3>(X, M, K, qw, qz, sc, gi, G, N, Y, s);
+    default: return launch_gemv<BITS, T, 4>(X, M, K, qw, qz, sc, gi, G, N, Y, s);
+  }
+}
+
 template <typename T>
 int gemv_any(int bits, const T* X, int M, int64_t K, const int32_t* qw, const int32_t* qz, const __half* sc,
              const int32_t* gi, int G, int64_t N, T* Y, cudaStream_t s) {
-  if (bits == 2) return launch_gemv<2, T>(X, M, K, qw, qz, sc, gi, G, N, Y, s);
-  if (bits == 4) return launch_gemv<4, T>(X, M, K, qw, qz, sc, gi, G, N, Y, s);
-  return launch_gemv<8, T>(X, M, K, qw, qz, sc, gi, G, N, Y, s);
+  if (bits == 2) return gemv_rows<2, T>(X, M, K, qw, qz, sc, gi, G, N, Y, s);
+  if (bits == 4) return gemv_rows<4, T>(X, M, K, qw, qz, sc, gi, G, N, Y, s);
+  return gemv_rows<8, T>(X, M, K, qw, qz, sc, gi, G, N, Y, s);
 }
 
 int check_qlinear(const int32_t* qweight, const int32_t* qzeros, const uint16_t* scales, const int32_t* g_idx,
