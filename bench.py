@@ -52,6 +52,10 @@ def parse_args():
     p.add_argument("--e2e-steps", type=int, default=6)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--two-phase", action="store_true",
+                   help="time the layer with factors and sweeps as two phases instead of the pipelined call")
+    p.add_argument("--phase-steps", type=int, default=3,
+                   help="untimed-for-the-headline two-phase steps that attribute time to the factor and the sweep")
     p.add_argument("--qlinear", action="store_true",
                    help="measure the linear on the quantized checkpoint (decode, dequantization, GEMM) alone")
     p.add_argument("--qlinear-shape", default="", help="with --qlinear: only the shapes whose name contains this")
@@ -220,8 +224,9 @@ def run_native(args, world, rank, local):
     Hbuf = {h: torch.empty(n, n, dtype=torch.float32, device=dev) for h, n in enumerate(cfg.hessian_n)}
     stream = torch.cuda.current_stream()
 
-    def step(timing=False):
-        return quantize_decoder_layer(acts, weights, cfg.layers, cfg, hessians=Hbuf, timing=timing, stream=stream)
+    def step(timing=False, pipelined=not args.two_phase):
+        return quantize_decoder_layer(acts, weights, cfg.layers, cfg, hessians=Hbuf, timing=timing, stream=stream,
+                                      pipelined=pipelined)
 
     for _ in range(max(args.warmup, 0)):
         step()
@@ -254,8 +259,19 @@ def run_native(args, world, rank, local):
     value = cols * world / (ms / 1e3)
     work = algorithmic_work(cfg, T)
     h_ms = statistics.mean(p.hessian_ms for p in phase)
-    f_ms = statistics.mean(p.factor_ms for p in phase)
-    s_ms = statistics.mean(p.sweep_ms for p in phase)
+    fs_ms = statistics.mean(p.factor_sweep_ms for p in phase)
+    spread = {"hessian_ms": [round(f(p.hessian_ms for p in phase), 3) for f in (min, statistics.median, max)],
+              "factor_and_sweep_ms": [round(f(p.factor_sweep_ms for p in phase), 3)
+                                      for f in (min, statistics.median, max)]}
+    # factor and sweep apart: the timed steps themselves in the two-phase route, else a few
+    # extra two-phase steps after the timed region (same inputs, bit-identical results)
+    attrib = phase
+    if not args.two_phase:
+        attrib = [step(timing=True, pipelined=False)[1] for _ in range(max(args.phase_steps, 1))]
+    f_ms = statistics.mean(p.factor_ms for p in attrib)
+    s_ms = statistics.mean(p.sweep_ms for p in attrib)
+    spread["two_phase_factor_ms"] = [round(f(p.factor_ms for p in attrib), 3) for f in (min, statistics.median, max)]
+    spread["two_phase_sweep_ms"] = [round(f(p.sweep_ms for p in attrib), 3) for f in (min, statistics.median, max)]
     launch_ms = [statistics.mean(p.hessian_launch_ms[i] for p in phase) for i in range(len(cfg.hessian_n))]
     h_flops = sum(work["hessian_flops"])
     h_tflops = h_flops / (sum(launch_ms) / 1e3) / 1e12
@@ -291,12 +307,17 @@ def run_native(args, world, rank, local):
                     "frac_of_datasheet_dense_bf16": round(h_tflops / DATASHEET_BF16_DENSE_TFLOPS, 4),
                     "datasheet_note": "2250 TFLOP/s: NVIDIA's dense (non-sparse) bf16 figure for B200 at its "
                                       "boost clock, not measured on this part"},
+        "factor_and_sweep": {"ms": round(fs_ms, 3), "pipelined": not args.two_phase,
+                             "two_phase_ms": round(f_ms + s_ms, 3),
+                             "note": "timed steps; factor and sweep below come from two-phase steps"
+                                     + ("" if args.two_phase else " run after the timed region")},
         "factor": {"ms": round(f_ms, 3), "tflops_fp64": round(f_tflops, 2),
                    "frac_of_fp64_peak": round(f_tflops / fp64_peak, 4)},
         "sweep": {"ms": round(s_ms, 3), "tflops_fp64": round(s_tflops, 2),
                   "frac_of_fp64_peak": round(s_tflops / fp64_peak, 4),
                   "min_hbm_gbs": round(work["sweep_min_bytes"] / (s_ms / 1e3) / 1e9, 1),
                   "frac_of_hbm": round(work["sweep_min_bytes"] / (s_ms / 1e3) / 1e9 / peaks["hbm"], 4)},
+        "spread_min_median_max": spread,
         "fp64_peak_tflops": round(fp64_peak, 1),
         "fp64_peak_how": "measured in this run: cuBLAS fp64 GEMM 8192^3 (torch.matmul), best of 3",
     }

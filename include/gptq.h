@@ -188,6 +188,41 @@ int gptq_quantize_layer_factored(const void* W, int w_dtype, int64_t n_out, int6
                                  int32_t* g_idx, void* stream, gptq_stats* stats);
 
 /*
+ * Factor once, sweep many, pipelined: every Hessian of a decoder layer factored and every
+ * linear that reads it quantized, in one call.  Source: chapter 5 §5.1.8 (factor U once per
+ * Hessian, then the column sweep of each weight against it) and the OLMo quick-start §六 6.1
+ * (modules that read the same input share one calibration Hessian).
+ *
+ * H[i], U[i], perm[i], n_in[i] (i < n_hessians): as in gptq_factor_hessians; U[i] and
+ *       perm[i] are outputs (the factor and sweep order of Hessian i, bit-identical to
+ *       gptq_factor_hessian's).
+ * W[j], n_out[j], qweight[j], scales[j], zeros[j], g_idx[j] (j < n_linears): one linear
+ *       each, laid out as in gptq_quantize_layer with n_in = n_in[hessian_of[j]];
+ *       hessian_of[j] names the Hessian of its input.  bits, group_size, sym,
+ *       static_groups, blocksize, w_dtype, damp_percent, desc_act: shared by all.
+ * Every output is bit-identical to gptq_factor_hessians followed by one
+ * gptq_quantize_layer_factored per linear (the same kernels in the same order per item).
+ * Scheduling: each Hessian's factor runs on its own library-owned stream (the largest at
+ * the highest priority) and each linear's sweep on its own stream, started as soon as its
+ * Hessian's factor is done, so the smaller Hessians' sweeps run while the largest factor is
+ * still in progress.  All streams fork from `stream` and join back into it.  Workspace
+ * (stream-ordered, from the library's pool): the factor workspaces of all Hessians plus
+ * 17 * n_out[j] * n_in bytes per linear, held until the call returns.
+ * statuses: optional host array of n_linears ints: the Hessian's factor status (NOT_PD)
+ * when that failed, else the linear's sweep status.  Returns GPTQ_OK when every linear
+ * succeeded, else the first failing linear's status.  n_hessians or n_linears <= 0, a NULL
+ * array or pointer, hessian_of out of range -> INVALID_ARG; argument rules of
+ * gptq_factor_hessians and gptq_quantize_layer otherwise.  Blocking.
+ */
+int gptq_quantize_linears(int n_hessians, const float* const* H, const int64_t* n_in,
+                          float damp_percent, int desc_act, double* const* U, int32_t* const* perm,
+                          int n_linears, const void* const* W, int w_dtype, const int64_t* n_out,
+                          const int* hessian_of, int bits, int group_size, int sym,
+                          int static_groups, int blocksize, int32_t* const* qweight,
+                          float* const* scales, int32_t* const* zeros, int32_t* const* g_idx,
+                          void* stream, int* statuses);
+
+/*
  * Checkpoint form of one quantized linear: half-precision scales and packed zero points.
  * Source: AutoGPTQ examples guide §1.4 and the OLMo quick-start §四 step 4
  * (save_quantized stores the quantized weights, with scale and zero point, beside

@@ -19,6 +19,7 @@ from .api import (  # noqa: F401
     launch_count,
     quantize_layer,
     quantize_layer_factored,
+    quantize_linears,
     quantized_linear,
 )
 

@@ -48,6 +48,12 @@ _SIGNATURES = {
     "gptq_quantize_layer_factored": (c_int, [c_void_p, c_int, c_i64, c_i64, c_void_p, c_void_p, c_int, c_int,
                                              c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
                                              c_void_p, ctypes.POINTER(GptqStats)]),
+    "gptq_quantize_linears": (c_int, [c_int, ctypes.POINTER(c_void_p), ctypes.POINTER(c_i64), c_float, c_int,
+                                      ctypes.POINTER(c_void_p), ctypes.POINTER(c_void_p), c_int,
+                                      ctypes.POINTER(c_void_p), c_int, ctypes.POINTER(c_i64), ctypes.POINTER(c_int),
+                                      c_int, c_int, c_int, c_int, c_int, ctypes.POINTER(c_void_p),
+                                      ctypes.POINTER(c_void_p), ctypes.POINTER(c_void_p), ctypes.POINTER(c_void_p),
+                                      c_void_p, ctypes.POINTER(c_int)]),
     "gptq_export_layer": (c_int, [c_void_p, c_void_p, c_i64, c_i64, c_int, c_void_p, c_void_p, c_void_p]),
     "gptq_dequantize_weight": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_i64, c_i64, c_i64, c_int, c_int,
                                        c_void_p, c_void_p]),

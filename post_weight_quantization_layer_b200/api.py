@@ -206,6 +206,55 @@ def quantize_layer_factored(W, U, perm, bits=4, group_size=128, sym=True, static
     return QuantResult(qw, sc, zr, gi, _stats_dict(st_obj) if stats else None)
 
 
+def quantize_linears(Hs, linears, bits=4, group_size=128, damp_percent=0.01, sym=True, desc_act=False,
+                      static_groups=False, blocksize=128, stream=None):
+    """Factor every Hessian in Hs and quantize every linear in one pipelined call.
+
+    Hs:      list of [n, n] float32 Hessians.
+    linears: list of (W, h) pairs: W [n_out, n_in] weight (all of one dtype) whose input has
+             Hessian Hs[h].
+    Returns ([(U, perm) per Hessian], [QuantResult per linear]): bit-identical to
+    factor_hessians followed by quantize_layer_factored per linear.  Raises GPTQError naming
+    the first linear that failed."""
+    Hs, linears = list(Hs), list(linears)
+    if not Hs or not linears:
+        raise ValueError("quantize_linears needs at least one Hessian and one linear")
+    for i, H in enumerate(Hs):
+        if not isinstance(H, torch.Tensor) or H.dim() != 2:
+            raise ValueError(f"H[{i}] must be a square 2-D tensor")
+        _need(H, f"H[{i}]", (torch.float32,), (H.shape[0], H.shape[0]))
+    dtypes = {W.dtype for W, _ in linears if isinstance(W, torch.Tensor)}
+    if len(dtypes) > 1:
+        raise ValueError("every linear must have the same weight dtype")
+    outs, hidx = [], []
+    for j, (W, h) in enumerate(linears):
+        if not isinstance(h, int) or not 0 <= h < len(Hs):
+            raise ValueError(f"linear {j}: Hessian index {h!r} out of range")
+        n_out, n_in = _weight(W)
+        if n_in != Hs[h].shape[0]:
+            raise ValueError(f"linear {j}: n_in {n_in} does not match its Hessian's order {Hs[h].shape[0]}")
+        outs.append(_outputs(n_out, n_in, bits, group_size, W.device, None))
+        hidx.append(h)
+    _need_cuda(*Hs, *[W for W, _ in linears])
+    factors = [(torch.empty(H.shape[0], H.shape[0], dtype=torch.float64, device=H.device),
+                torch.empty(H.shape[0], dtype=torch.int32, device=H.device)) for H in Hs]
+    kh, kl = len(Hs), len(linears)
+    ah, al = ctypes.c_void_p * kh, ctypes.c_void_p * kl
+    st_arr = (ctypes.c_int * kl)()
+    st = lib().gptq_quantize_linears(
+        kh, ah(*[H.data_ptr() for H in Hs]), (ctypes.c_int64 * kh)(*[H.shape[0] for H in Hs]), float(damp_percent),
+        int(bool(desc_act)), ah(*[U.data_ptr() for U, _ in factors]), ah(*[p.data_ptr() for _, p in factors]), kl,
+        al(*[W.data_ptr() for W, _ in linears]), _DTYPE.get(linears[0][0].dtype, 99),
+        (ctypes.c_int64 * kl)(*[W.shape[0] for W, _ in linears]), (ctypes.c_int * kl)(*hidx), bits, group_size,
+        int(bool(sym)), int(bool(static_groups)), blocksize, al(*[o[0].data_ptr() for o in outs]),
+        al(*[o[1].data_ptr() for o in outs]), al(*[o[2].data_ptr() for o in outs]),
+        al(*[o[3].data_ptr() for o in outs]), _stream(stream), st_arr)
+    if st != OK:
+        bad = next((j for j in range(kl) if st_arr[j] != OK), None)
+        _check(st, "gptq_quantize_linears" + (f" (linear {bad})" if bad is not None else ""))
+    return factors, [QuantResult(*o, None) for o in outs]
+
+
 def _checkpoint(ck, bits):
     """(qweight, qzeros, scales, g_idx, groups, n_in, n_out) of a checkpoint-form linear
     (the dict of export.export_layer / export.load_quantized), checked."""

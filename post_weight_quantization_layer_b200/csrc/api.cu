@@ -3,6 +3,7 @@
 #include <cstring>
 #include <map>
 #include <mutex>
+#include <memory>
 #include <vector>
 
 #include "common.cuh"
@@ -353,6 +354,99 @@ int gptq_factor_hessians(int count, const float* const* H, const int64_t* n_in, 
   for (int i = 0; i < count; ++i) {
     if (statuses) statuses[i] = h[static_cast<size_t>(i)];
     if (first == GPTQ_OK && h[static_cast<size_t>(i)] != GPTQ_OK) first = h[static_cast<size_t>(i)];
+  }
+  return first;
+}
+
+int gptq_quantize_linears(int n_hessians, const float* const* H, const int64_t* n_in, float damp_percent,
+                          int desc_act, double* const* U, int32_t* const* perm, int n_linears,
+                          const void* const* W, int w_dtype, const int64_t* n_out, const int* hessian_of, int bits,
+                          int group_size, int sym, int static_groups, int blocksize, int32_t* const* qweight,
+                          float* const* scales, int32_t* const* zeros, int32_t* const* g_idx, void* stream,
+                          int* statuses) {
+  if (n_hessians <= 0 || n_linears <= 0 || !H || !n_in || !U || !perm || !W || !n_out || !hessian_of || !qweight ||
+      !scales || !zeros || !g_idx)
+    return GPTQ_ERR_INVALID_ARG;
+  if (!valid_damp(damp_percent)) return GPTQ_ERR_INVALID_ARG;
+  for (int i = 0; i < n_hessians; ++i) {
+    if (!H[i] || !U[i] || !perm[i] || n_in[i] <= 0) return GPTQ_ERR_INVALID_ARG;
+    if (n_in[i] % 8 != 0 || n_in[i] > 65535) return GPTQ_ERR_UNSUPPORTED;
+    if (!aligned16(H[i]) || !aligned16(U[i]) || !aligned16(perm[i])) return GPTQ_ERR_UNSUPPORTED;
+  }
+  for (int j = 0; j < n_linears; ++j) {
+    if (hessian_of[j] < 0 || hessian_of[j] >= n_hessians) return GPTQ_ERR_INVALID_ARG;
+    GPTQ_TRY(check_quant_args(W[j], w_dtype, n_out[j], n_in[hessian_of[j]], bits, group_size, blocksize, qweight[j],
+                              scales[j], zeros[j], g_idx[j]));
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  size_t bytes = padded(static_cast<size_t>(n_hessians + n_linears) * sizeof(int));
+  for (int i = 0; i < n_hessians; ++i)
+    bytes += padded(factor_work_bytes(n_in[i], true)) + padded(factor_small_bytes(n_in[i])) +
+             padded(static_cast<size_t>(n_in[i]) * 4);
+  for (int j = 0; j < n_linears; ++j) {
+    const size_t e = static_cast<size_t>(n_out[j]) * static_cast<size_t>(n_in[hessian_of[j]]);
+    bytes += 2 * padded(e * 8) + padded(e) + padded(sizeof(double));
+  }
+  Workspace ws;  // declared before the leases: freed on s after every lane has joined
+  GPTQ_TRY(alloc(ws, bytes + 256, s));
+  int* dstat = ws.take<int>(static_cast<size_t>(n_hessians + n_linears));
+  GPTQ_CUDA(cudaMemsetAsync(dstat, 0, static_cast<size_t>(n_hessians + n_linears) * sizeof(int), s));
+  int largest = 0;
+  for (int i = 1; i < n_hessians; ++i)
+    if (n_in[i] > n_in[largest]) largest = i;
+  std::vector<LanePrio> prio(static_cast<size_t>(n_hessians), kLaneLow);
+  prio[static_cast<size_t>(largest)] = kLaneHigh;
+  std::vector<int32_t*> invperm(static_cast<size_t>(n_hessians), nullptr);
+  Events off;
+  GPTQ_TRY(off.create(false));
+  {
+    // One chain lane per Hessian: its factor, then (forked from it) one lane per linear
+    // that reads it.  The sub-leases end before the chain lease (reverse declaration order).
+    LaneLease chains(s);
+    GPTQ_TRY(chains.acquire(n_hessians, prio.data()));
+    std::vector<std::unique_ptr<LaneLease>> subs;
+    for (int i = 0; i < n_hessians; ++i) {
+      const int64_t n = n_in[i];
+      void* work = ws.take<char>(factor_work_bytes(n, true));
+      void* small = ws.take<char>(factor_small_bytes(n));
+      invperm[static_cast<size_t>(i)] = ws.take<int32_t>(static_cast<size_t>(n));
+      GPTQ_TRY(factor_on_lanes(H[i], n, damp_percent, desc_act != 0, U[i], perm[i], invperm[static_cast<size_t>(i)],
+                               work, small, dstat + i, true, prio[static_cast<size_t>(i)], chains[i].st));
+    }
+    for (int i = 0; i < n_hessians; ++i) {
+      std::vector<int> mine;
+      for (int j = 0; j < n_linears; ++j)
+        if (hessian_of[j] == i) mine.push_back(j);
+      if (mine.empty()) continue;
+      subs.emplace_back(new LaneLease(chains[i].st));
+      LaneLease& lease = *subs.back();
+      const std::vector<LanePrio> lp(mine.size(), prio[static_cast<size_t>(i)]);
+      GPTQ_TRY(lease.acquire(static_cast<int>(mine.size()), lp.data()));
+      const int64_t ni = n_in[i];
+      for (size_t t = 0; t < mine.size(); ++t) {
+        const int j = mine[t];
+        const size_t e = static_cast<size_t>(n_out[j]) * static_cast<size_t>(ni);
+        double* Wk = ws.take<double>(e);
+        double* Err = ws.take<double>(e);
+        uint8_t* codesT = ws.take<uint8_t>(e);
+        double* loss = ws.take<double>(1);
+        GPTQ_TRY(sweep_common(W[j], w_dtype, n_out[j], ni, U[i], desc_act ? perm[i] : nullptr,
+                              desc_act ? invperm[static_cast<size_t>(i)] : nullptr, bits, group_size, sym,
+                              static_groups, blocksize, qweight[j], scales[j], zeros[j], g_idx[j], Wk, Err, codesT,
+                              loss, dstat + n_hessians + j, lease[static_cast<int>(t)].st, nullptr, off, 0));
+      }
+    }
+  }  // every lane joins back into s
+  std::vector<int> h(static_cast<size_t>(n_hessians + n_linears), 0);
+  if (cudaMemcpyAsync(h.data(), dstat, h.size() * sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return GPTQ_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return GPTQ_ERR_CUDA;
+  int first = GPTQ_OK;
+  for (int j = 0; j < n_linears; ++j) {
+    const int hf = h[static_cast<size_t>(hessian_of[j])];
+    const int st = hf != GPTQ_OK ? hf : h[static_cast<size_t>(n_hessians + j)];
+    if (statuses) statuses[j] = st;
+    if (first == GPTQ_OK && st != GPTQ_OK) first = st;
   }
   return first;
 }

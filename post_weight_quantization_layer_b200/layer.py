@@ -2,11 +2,15 @@
 
 The modules that read the same input share one calibration Hessian (q/k/v the
 attention input, gate/up the MLP input; the OLMo quick-start's fused att_proj,
-§六 6.1).  Each distinct Hessian is accumulated once, factored once (all of them
-in one gptq_factor_hessians call, which runs them concurrently), and every module
-that reads it is swept against that factor (gptq_quantize_layer_factored).  All arithmetic runs in the native
-library; this module only sequences the calls and records per-phase CUDA-event
-times on the stream.
+§六 6.1).  Each distinct Hessian is accumulated once and factored once, and every
+module that reads it is swept against that factor.  By default the factors and
+sweeps are one pipelined native call (gptq_quantize_linears: each linear's sweep
+starts as soon as its own Hessian is factored, while the larger factors are still
+running); pipelined=False runs them as two phases (gptq_factor_hessians, then one
+gptq_quantize_layer_factored per module), which gives bit-identical results and
+separate factor and sweep times.  All arithmetic runs in the native library; this
+module only sequences the calls and records per-phase CUDA-event times on the
+stream.
 """
 
 from __future__ import annotations
@@ -21,17 +25,18 @@ from . import api
 @dataclass
 class LayerTimes:
     hessian_ms: float = 0.0
-    factor_ms: float = 0.0
-    sweep_ms: float = 0.0
+    factor_ms: float = 0.0  # two-phase route only
+    sweep_ms: float = 0.0  # two-phase route only
+    factor_sweep_ms: float = 0.0  # factors and sweeps together (both routes)
     hessian_launch_ms: list = field(default_factory=list)
 
     @property
     def total_ms(self):
-        return self.hessian_ms + self.factor_ms + self.sweep_ms
+        return self.hessian_ms + self.factor_sweep_ms
 
 
 def quantize_decoder_layer(acts, weights, modules, qcfg, hessians=None, timing=False, stream=None,
-                           hessians_given=False):
+                           hessians_given=False, pipelined=True):
     """Quantize the linears of one decoder layer.
 
     acts:     {h_index: X [tokens, n] fp16/bf16 CUDA tensor, or a list of token chunks}
@@ -42,6 +47,7 @@ def quantize_decoder_layer(acts, weights, modules, qcfg, hessians=None, timing=F
     hessians_given: the `hessians` already hold the layer's Hessians (accumulated earlier,
               e.g. streamed chunk by chunk); `acts` is then ignored and nothing is
               accumulated.
+    pipelined: factors and sweeps in one overlapped call (default) or as two phases.
     Returns ({module name: QuantResult}, LayerTimes or None).
     """
     stream = stream or torch.cuda.current_stream()
@@ -77,22 +83,33 @@ def quantize_decoder_layer(acts, weights, modules, qcfg, hessians=None, timing=F
             launch_marks.append((a, b))
             Hs[h] = H
         m_h = mark()
-        # every distinct Hessian factored in one call: the library runs them concurrently
         keys = list(Hs)
-        factors = dict(zip(keys, api.factor_hessians([Hs[h] for h in keys], qcfg.damp_percent, qcfg.desc_act,
-                                                     stream=stream)))
-        m_f = mark()
-        results = {}
-        for mod in modules:
-            U, perm = factors[mod.h_index]
-            results[mod.name] = api.quantize_layer_factored(
-                weights[mod.name], U, perm, qcfg.bits, qcfg.group_size, qcfg.sym, qcfg.static_groups,
-                qcfg.blocksize, stream=stream)
+        m_f = None
+        if pipelined:
+            hpos = {h: i for i, h in enumerate(keys)}
+            mods = list(modules)
+            _, res = api.quantize_linears([Hs[h] for h in keys], [(weights[m.name], hpos[m.h_index]) for m in mods],
+                                          qcfg.bits, qcfg.group_size, qcfg.damp_percent, qcfg.sym, qcfg.desc_act,
+                                          qcfg.static_groups, qcfg.blocksize, stream=stream)
+            results = {m.name: r for m, r in zip(mods, res)}
+        else:
+            # every distinct Hessian factored in one call: the library runs them concurrently
+            factors = dict(zip(keys, api.factor_hessians([Hs[h] for h in keys], qcfg.damp_percent, qcfg.desc_act,
+                                                         stream=stream)))
+            m_f = mark()
+            results = {}
+            for mod in modules:
+                U, perm = factors[mod.h_index]
+                results[mod.name] = api.quantize_layer_factored(
+                    weights[mod.name], U, perm, qcfg.bits, qcfg.group_size, qcfg.sym, qcfg.static_groups,
+                    qcfg.blocksize, stream=stream)
         m_s = mark()
     if timing:
         m_s.synchronize()
         times.hessian_ms = marks[0].elapsed_time(m_h)
-        times.factor_ms = m_h.elapsed_time(m_f)
-        times.sweep_ms = m_f.elapsed_time(m_s)
+        times.factor_sweep_ms = m_h.elapsed_time(m_s)
+        if m_f is not None:
+            times.factor_ms = m_h.elapsed_time(m_f)
+            times.sweep_ms = m_f.elapsed_time(m_s)
         times.hessian_launch_ms = [a.elapsed_time(b) for a, b in launch_marks]
     return results, times

@@ -51,12 +51,11 @@ def _quantize_group(X, names, weights, qcfg, stream):
     n = X.shape[1]
     H = torch.zeros(n, n, dtype=torch.float32, device=X.device)
     api.accumulate_hessian(X, H, stream=stream)
-    U, perm = api.factor_hessian(H, qcfg.damp_percent, qcfg.desc_act, stream=stream)
-    out = {}
-    for name in names:
-        out[name] = api.quantize_layer_factored(weights[name], U, perm, qcfg.bits, qcfg.group_size, qcfg.sym,
-                                                qcfg.static_groups, qcfg.blocksize, stream=stream)
-    return out
+    # one factor, the group's sweeps side by side (gptq_quantize_linears)
+    _, res = api.quantize_linears([H], [(weights[name], 0) for name in names], qcfg.bits, qcfg.group_size,
+                                  qcfg.damp_percent, qcfg.sym, qcfg.desc_act, qcfg.static_groups, qcfg.blocksize,
+                                  stream=stream)
+    return dict(zip(names, res))
 
 
 def quantize_decoder_layer_sequential(h, weights, gammas, shape: DecoderShape, qcfg, given=None, given_inputs=None,

@@ -143,3 +143,53 @@ def test_odd_group_sizes(n_out, n_in, g):
     W, H = _problem(n_out, n_in, 8 * n_in, n_in + g, w_dtype=torch.float32)
     _, _, m = _run(W, H, 4, g, False, False, False)
     assert_parity(m, (n_out, n_in, g))
+
+
+@pytest.mark.parametrize("desc_act", [False, True])
+def test_pipelined_linears_equal_factor_then_sweeps(desc_act):
+    """quantize_linears (each Hessian's factor on its own stream, each linear's sweep started
+    when its factor is done) gives exactly the factors of factor_hessians and the codes of one
+    quantize_layer_factored per linear; one linear is also checked against the oracle."""
+    dev = device()
+    shapes = [(512, 2048, 61), (256, 1024, 62), (1024, 4096, 63)]
+    Hs, Ws = [], []
+    for n, T, seed in shapes:
+        W, H = _problem(8, n, T, seed)
+        Hs.append(H.to(dev))
+    lin = [(synth.outlier_weight(96, 512, 70), 0), (synth.outlier_weight(40, 256, 71), 1),
+           (synth.outlier_weight(64, 512, 72), 0), (synth.outlier_weight(200, 1024, 73), 2),
+           (synth.outlier_weight(24, 1024, 74), 2)]
+    lin = [(W.to(dev), h) for W, h in lin]
+    factors, res = gq.quantize_linears(Hs, lin, 4, 32, 0.01, True, desc_act, desc_act, 128)
+    torch.cuda.synchronize()
+    ref_f = gq.factor_hessians(Hs, 0.01, desc_act)
+    for (U, p), (U1, p1) in zip(factors, ref_f):
+        assert torch.equal(p, p1)
+        assert torch.equal(U, U1)
+    for (W, h), r in zip(lin, res):
+        U1, p1 = ref_f[h]
+        b = gq.quantize_layer_factored(W, U1, p1, 4, 32, True, desc_act, 128)
+        for x, y in zip((r.qweight, r.scales, r.zeros, r.g_idx), (b.qweight, b.scales, b.zeros, b.g_idx)):
+            assert torch.equal(x, y)
+    W, h = lin[3]
+    Wn, Hn = W.double().cpu().numpy(), Hs[h].double().cpu().numpy()
+    ref = O.gptq_quantize(Wn, Hn, 4, 32, 0.01, True, desc_act, desc_act)
+    assert_parity(compare_quant(res[3], ref, Wn, Hn, 4, 1024), "pipelined")
+
+
+def test_pipelined_linears_report_the_failing_linear():
+    dev = device()
+    _, good = _problem(8, 256, 1024, 81)
+    good = good.to(dev)
+    bad = -torch.eye(128, device=dev)
+    lin = [(synth.outlier_weight(32, 256, 82).to(dev), 0), (torch.randn(16, 128, device=dev).half(), 1)]
+    with pytest.raises(gq.GPTQError) as e:
+        gq.quantize_linears([good, bad], lin, 4, 32, 0.01, True, True)
+    assert e.value.status == 3 and "linear 1" in str(e.value)
+    with pytest.raises(ValueError):
+        gq.quantize_linears([good], [(lin[0][0], 1)], 4, 32)
+    # the context stays usable and the good Hessian's linear matches the two-call route
+    factors, res = gq.quantize_linears([good], lin[:1], 4, 32, 0.01, True, True)
+    U1, p1 = gq.factor_hessian(good, 0.01, True)
+    b = gq.quantize_layer_factored(lin[0][0], U1, p1, 4, 32, True, False, 128)
+    assert torch.equal(res[0].qweight, b.qweight)
