@@ -53,6 +53,14 @@ constexpr uint32_t IWAIT = 1u << 24;
 
 __device__ int g_i8_status = 0;
 
+// 2^e as a double: built from the exponent bits in the normal range, else by ldexp.
+__device__ __forceinline__ double pow2(int e) {
+  if (e >= -1022 && e <= 1023) return __longlong_as_double(static_cast<long long>(e + 1023) << 52);
+  return ldexp(1.0, e);
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
 // ------------------------------------------------------------------ splitting
 // One warp per row of A (rows of Err[:, block], K = block width): the row exponent, then
 // KS slices of every element.  S is [KS][R][KP] (k contiguous, zero padded to KP).
@@ -306,9 +314,21 @@ __global__ void __maxnreg__(160)
     // owns one column n (its TMEM lane); the 4 warps of each lane quarter are split over the
     // tile's 48 rows in chunks of 16 (warps 2..5 and 6..9 take chunks 0, 2 and 1); for each
     // row the warp's 32 lanes update 32 consecutive columns (coalesced).  The 16 loads of W are
-    // issued together before any use.
+    // issued together before any use, and the rows of this CTA's next tile are prefetched into
+    // L2 while the current one is updated.
     const int quad = warp & 3;
     const int half = (warp - 2) >> 2;
+    const int et = threadIdx.x - 64;  // 0..255 over the epilogue warps
+    // L2 prefetch of the W lines (48 rows x 1 KiB) of tile u: 384 lines of 128 bytes
+    auto prefetch_tile = [&](int u) {
+      if (u >= units) return;
+      const int cb = (u / a.mt) * IBM, rb = (u % a.mt) * IBN;
+      for (int l = et; l < IBN * (IBM / 16); l += 256) {
+        const int r = rb + l / (IBM / 16), cc = cb + (l % (IBM / 16)) * 16;
+        if (r < a.M && cc < a.N) prefetch_l2(a.C + static_cast<int64_t>(r) * a.ldc + cc);
+      }
+    };
+    prefetch_tile(blockIdx.x);
     int cg = 0;
     for (int u = blockIdx.x; u < units; u += G, ++cg) {
       const int b = cg & 1;
@@ -317,9 +337,12 @@ __global__ void __maxnreg__(160)
         break;
       }
       tc_fence_after();
+      prefetch_tile(u + G);
       const int c = (u / a.mt) * IBM + quad * 32 + lane;  // column within this launch
       const bool cin = c < a.N;
-      const int ec = cin ? a.eb[a.col0 + c] - 2 * SBETA : 0;
+      // 2^(eb_n - 14 - 28): the column's share of the scale, with the 2^-28 that turns the
+      // integer recombination below into sum_s acc_s 2^(-7 s)
+      const int ec = cin ? a.eb[a.col0 + c] - 2 * SBETA - (KS - 1) * SBETA : 0;
       for (int chunk = half; chunk < IBN / 16; chunk += 2) {
         const int r0 = (u % a.mt) * IBN + chunk * 16;
         int acc[KS][16];
@@ -334,10 +357,13 @@ __global__ void __maxnreg__(160)
           cv[j] = (cin && r0 + j < a.M) ? a.C[static_cast<int64_t>(r0 + j) * a.ldc + c] : 0.0;
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          double v = static_cast<double>(acc[KS - 1][j]);
+          // sum_s acc_s 2^(7 (KS-1-s)) exactly in 64-bit integers (|acc_s| < 2^31, so the sum
+          // stays below 2^60), then one rounding to fp64 and an exact power-of-two scale
+          long long v = acc[0][j];
 #pragma unroll
-          for (int s = KS - 2; s >= 0; --s) v = fma(v, 0x1p-7, static_cast<double>(acc[s][j]));
-          if (cin && r0 + j < a.M) a.C[static_cast<int64_t>(r0 + j) * a.ldc + c] = cv[j] - ldexp(v, ec + a.ea[r0 + j]);
+          for (int s = 1; s < KS; ++s) v = v * (1ll << SBETA) + acc[s][j];
+          if (cin && r0 + j < a.M)
+            a.C[static_cast<int64_t>(r0 + j) * a.ldc + c] = cv[j] - static_cast<double>(v) * pow2(ec + a.ea[r0 + j]);
         }
       }
       tc_fence_before();

@@ -27,7 +27,7 @@
 //   left-looking product on the fp64 matrix units); after each outer block its errors
 //   update every later column at once.  That trailing update runs on the int8 tensor cores
 //   (ozaki.cu: both operands split into five 7-bit slices, exact integer slice products,
-//   fp64 recombination), which leaves the fp64 pipe to the panels' compensation chain.
+//   exact integer recombination), which leaves the fp64 pipe to the panels' compensation chain.
 // * Look-ahead: the trailing update is split in two.  The next outer block's columns are
 //   updated first, on a high-priority stream that then runs the next block's panels; the
 //   rest runs at the same time on a low-priority stream.  A panel CTA and a trailing-update
