@@ -98,6 +98,12 @@ int i8_split_cols(cudaStream_t s, const double* Y, int64_t ldy, int64_t K, int64
 int i8_gemm_sub(cudaStream_t s, int64_t M, int64_t N, int64_t KP, const int8_t* SA, int64_t a_rows, const int* ea,
                 const int8_t* SB, int64_t b_cols, const int* eb, int64_t col0, double* C, int64_t ldc,
                 int max_ctas);
+int i8f_slices();
+int i8f_split_rows(cudaStream_t s, const double* X, int64_t ldx, int64_t R, int64_t K, int64_t KP, int8_t* S, int* e);
+int i8f_split_cols(cudaStream_t s, const double* Y, int64_t ldy, int64_t K, int64_t N, int64_t KP, int8_t* S,
+                   int* e);
+int i8f_gemm_sub(cudaStream_t s, int64_t M, int64_t N, int64_t KP, const int8_t* SA, int64_t a_rows, const int* ea,
+                 const int8_t* SB, int64_t b_cols, const int* eb, double* C, int64_t ldc, int krange, int upper);
 int i8_device_status(int clear);
 
 // factor.cu: U (sweep order, fp64) and perm from H, stream-ordered on s.  `work` holds

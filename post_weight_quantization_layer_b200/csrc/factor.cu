@@ -297,41 +297,79 @@ int64_t right_part(int64_t n) {
   return std::min<int64_t>(n - 1, ((half + NB - 1) / NB) * NB);
 }
 
-// Largest P (n1 x n2) over all nodes, and largest T per recursion depth.
-void plan(int64_t n, int depth, size_t& pmax, std::vector<size_t>& tmax) {
+// Nodes whose right part is at least I8_MIN wide run their four products on the int8
+// tensor cores (seven-slice operands: 49 bits each, see ozaki.cu); smaller ones on the fp64
+// matrix units.  Both K of a node's products (n2 and n1) stay within the int8 kernel's 16384.
+constexpr int64_t I8_MIN = 1024;
+constexpr int64_t I8_MAX = 16384;
+bool node_i8(int64_t n2) { return n2 >= I8_MIN && n2 <= I8_MAX; }
+
+int64_t pad64(int64_t k) { return (k + 63) / 64 * 64; }
+
+struct Plan {
+  size_t pmax = 0;
+  std::vector<size_t> tmax;            // T per depth
+  std::vector<size_t> sx, sy, ex, ey;  // int8 slices (bytes) and exponents per depth
+};
+
+// Largest P (n1 x n2) over all nodes, and per recursion depth the largest T and int8 slice
+// buffers: X [KSF][n1][pad(n2)] (rows of B, then of P, then of U11), Y [KSF][n2][pad(n2)]
+// (rows of U22, then its columns, then the columns of T).
+void plan(int64_t n, int depth, Plan& pl) {
   if (n <= NB) return;
   const int64_t n2 = right_part(n), n1 = n - n2;
   const size_t sz = static_cast<size_t>(n1) * n2;
-  pmax = std::max(pmax, sz);
-  if (static_cast<int>(tmax.size()) <= depth) tmax.resize(depth + 1, 0);
-  tmax[depth] = std::max(tmax[depth], sz);
-  plan(n2, depth + 1, pmax, tmax);
-  plan(n1, depth + 1, pmax, tmax);
+  pl.pmax = std::max(pl.pmax, sz);
+  const size_t d = static_cast<size_t>(depth);
+  for (auto* v : {&pl.tmax, &pl.sx, &pl.sy, &pl.ex, &pl.ey})
+    if (v->size() <= d) v->resize(d + 1, 0);
+  pl.tmax[d] = std::max(pl.tmax[d], sz);
+  if (node_i8(n2)) {
+    const size_t ks = static_cast<size_t>(i8f_slices());
+    pl.sx[d] = std::max(pl.sx[d], ks * n1 * pad64(n2));
+    pl.sy[d] = std::max(pl.sy[d], ks * n2 * pad64(n2));
+    pl.ex[d] = std::max(pl.ex[d], static_cast<size_t>(n1));
+    pl.ey[d] = std::max(pl.ey[d], static_cast<size_t>(n2));
+  }
+  plan(n2, depth + 1, pl);
+  plan(n1, depth + 1, pl);
 }
 
 struct Scratch {
   real* P;
   real* P0;  // the top level's own P when its T product overlaps the left recursion
   std::vector<real*> T;
+  std::vector<int8_t*> SX, SY;
+  std::vector<int*> EX, EY;
 };
 
 size_t scratch_elems(int64_t n, Scratch* out, real* base, bool overlap) {
-  size_t pmax = 0;
-  std::vector<size_t> tmax;
-  plan(n, 0, pmax, tmax);
+  Plan pl;
+  plan(n, 0, pl);
   size_t off = 0;
   auto take = [&](size_t e) {
     real* p = base ? base + off : nullptr;
     off += (e + 31) & ~size_t(31);
     return p;
   };
-  real* P = take(pmax);
+  auto take_bytes = [&](size_t b) { return reinterpret_cast<char*>(take((b + sizeof(real) - 1) / sizeof(real))); };
+  real* P = take(pl.pmax);
   if (out) out->P = P;
-  real* P0 = (overlap && !tmax.empty()) ? take(tmax[0]) : nullptr;
+  real* P0 = (overlap && !pl.tmax.empty()) ? take(pl.tmax[0]) : nullptr;
   if (out) out->P0 = P0;
-  for (size_t d = 0; d < tmax.size(); ++d) {
-    real* t = take(tmax[d]);
-    if (out) out->T.push_back(t);
+  for (size_t d = 0; d < pl.tmax.size(); ++d) {
+    real* t = take(pl.tmax[d]);
+    int8_t* sx = pl.sx[d] ? reinterpret_cast<int8_t*>(take_bytes(pl.sx[d])) : nullptr;
+    int8_t* sy = pl.sy[d] ? reinterpret_cast<int8_t*>(take_bytes(pl.sy[d])) : nullptr;
+    int* ex = pl.ex[d] ? reinterpret_cast<int*>(take_bytes(pl.ex[d] * sizeof(int))) : nullptr;
+    int* ey = pl.ey[d] ? reinterpret_cast<int*>(take_bytes(pl.ey[d] * sizeof(int))) : nullptr;
+    if (out) {
+      out->T.push_back(t);
+      out->SX.push_back(sx);
+      out->SY.push_back(sy);
+      out->EX.push_back(ex);
+      out->EY.push_back(ey);
+    }
   }
   return off;
 }
@@ -358,12 +396,42 @@ int factor_rec(real* A, real* R, int64_t n, int64_t lo, int64_t hi, int depth, S
   const bool overlap = depth == 0 && ov.side != nullptr && sc.P0 != nullptr;
   real* P = overlap ? sc.P0 : sc.P;
   real* T = sc.T[depth];
+  const size_t d = static_cast<size_t>(depth);
+  const bool i8 = node_i8(n2);
+  cudaStream_t st = s;
+  if (i8) {
+    // Int8 route, in negated form so that every product is a subtraction C -= A B:
+    //   P' = 0 - B U22^T = -P;  A' = A - P' P'^T;  T = 0 - P' U22 = P U22;  U12 = 0 - U11 T.
+    int8_t *SX = sc.SX[d], *SY = sc.SY[d];
+    int *EX = sc.EX[d], *EY = sc.EY[d];
+    const int64_t K2 = pad64(n2), K1 = pad64(n1);
+    GPTQ_TRY(i8f_split_rows(s, A + lo * n + mid, n, n1, n2, K2, SX, EX));
+    GPTQ_TRY(i8f_split_rows(s, U22, n, n2, n2, K2, SY, EY));
+    GPTQ_CUDA(cudaMemsetAsync(P, 0, static_cast<size_t>(n1) * n2 * sizeof(real), s));
+    GPTQ_TRY(i8f_gemm_sub(s, n1, n2, K2, SX, n1, EX, SY, n2, EY, P, n2, /*B[k, c] = U22[c, k]*/ 1, 0));
+    GPTQ_TRY(i8f_split_rows(s, P, n2, n1, n2, K2, SX, EX));
+    GPTQ_TRY(i8f_gemm_sub(s, n1, n1, K2, SX, n1, EX, SX, n1, EX, A + lo * n + lo, n, 0, /*upper*/ 1));
+    if (overlap) {
+      GPTQ_CUDA(cudaEventRecord(ov.p_ready, s));
+      GPTQ_CUDA(cudaStreamWaitEvent(ov.side, ov.p_ready, 0));
+      st = ov.side;
+    }
+    GPTQ_TRY(i8f_split_cols(st, U22, n, n2, n2, K2, SY, EY));
+    GPTQ_CUDA(cudaMemsetAsync(T, 0, static_cast<size_t>(n1) * n2 * sizeof(real), st));
+    GPTQ_TRY(i8f_gemm_sub(st, n1, n2, K2, SX, n1, EX, SY, n2, EY, T, n2, /*B[k, c] = U22[k, c]*/ 2, 0));
+    if (overlap) GPTQ_CUDA(cudaEventRecord(ov.t_ready, ov.side));
+    GPTQ_TRY(factor_rec(A, R, n, lo, mid, depth + 1, sc, status, s, ov));
+    if (overlap) GPTQ_CUDA(cudaStreamWaitEvent(s, ov.t_ready, 0));
+    GPTQ_TRY(i8f_split_rows(s, R + lo * n + lo, n, n1, n1, K1, SX, EX));
+    GPTQ_TRY(i8f_split_cols(s, T, n2, n1, n2, K1, SY, EY));
+    // U12 starts at zero (U is cleared before the recursion)
+    return i8f_gemm_sub(s, n1, n2, K1, SX, n1, EX, SY, n2, EY, R + lo * n + mid, n, /*A[r, k] = U11[r, k]*/ 3, 0);
+  }
   // P = B U22^T
   GPTQ_TRY(dgemm(s, n1, n2, n2, 1.0, A + lo * n + mid, n, U22, n, true, 0.0, P, n2, false, kTriBTUpper));
   // A' = A - P P^T (upper tiles)
   GPTQ_TRY(dgemm(s, n1, n1, n2, -1.0, P, n2, P, n2, true, 1.0, A + lo * n + lo, n, true));
   // T = P U22
-  cudaStream_t st = s;
   if (overlap) {
     GPTQ_CUDA(cudaEventRecord(ov.p_ready, s));
     GPTQ_CUDA(cudaStreamWaitEvent(ov.side, ov.p_ready, 0));

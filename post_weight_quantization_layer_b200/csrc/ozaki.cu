@@ -1,4 +1,5 @@
-// The sweep's lazy trailing update on the 5th-generation int8 tensor cores.
+// fp64-accurate matrix products on the 5th-generation int8 tensor cores: the sweep's lazy
+// trailing update, and the large products of the recursive factorisation.
 //
 // Source of the operation: "第5章 GPTQ 实战" §5.1.8 key point 3 (lazy batch update): after a
 // block of columns is quantized, its normalised errors update every later column at once,
@@ -17,15 +18,25 @@
 //   bits, left a few more near-tie flips than fp64 in the parity tests).  Each SA_p SB_q^T
 //   is an exact int32 product (127^2 * K * 5 < 2^31 for K <= 16384).
 //
+// The factorisation ("第5章 GPTQ 实战" §5.1.8 key point 1, the inverse-Cholesky factor U)
+// uses the same scheme with seven slices per operand (49 bits; the 28 pairs p + q <= 6,
+// 7 * 127^2 * K < 2^31 for K <= 16384): its Schur complements cancel, so it keeps more bits
+// than the sweep needs.
+//
 // Kernels: split_rows_kernel / split_cols_kernel write the slices K-major (k contiguous)
-// for TMA; i8_gemm_kernel runs tcgen05.mma kind::i8 (s8 x s8 -> s32) with the U slices as
-// the M side (128 later columns) and the Err slices as the N side (48 rows of W), five TMEM
-// accumulators (one per s = p + q), double buffered, a 2-stage TMA ring of all slices of a
-// 64-wide K step (64-byte swizzle).  Its 111 KB of shared memory and 160 registers a thread
-// leave room on the SM for one CTA of the sweep's panel kernel, which runs beside it.  In
-// the epilogue a thread owns one column and a warp updates 32 consecutive columns of a row
-// at a time (coalesced fp64 read-modify-write, loads issued together); each element of W is
-// updated by exactly one thread of one CTA per launch (deterministic).
+// for TMA; i8_gemm_kernel<NS, BN, NBUF, CR> runs tcgen05.mma kind::i8 (s8 x s8 -> s32) with
+// the column operand's slices as the M side (128 columns of C) and the row operand's as the
+// N side (BN rows of C), NS TMEM accumulators (one per s = p + q), NBUF accumulator
+// buffers, a 2-stage TMA ring of all slices of a 64-wide K step (64-byte swizzle).
+//  * sweep: 5 slices, 48 rows, double buffered: 111 KB of shared memory and 160 registers
+//    a thread leave room on the SM for one CTA of the sweep's panel kernel, which runs
+//    beside it.
+//  * factor: 7 slices, 64 rows, one buffer (448 TMEM columns; 172 KB of shared memory);
+//    a tile may skip the K steps where a triangular operand is zero, and a symmetric
+//    update may skip the tiles strictly below the diagonal.
+// In the epilogue a thread owns one column and a warp updates 32 consecutive columns of a
+// row at a time (coalesced fp64 read-modify-write, loads issued together); each element of
+// C is updated by exactly one thread of one CTA per launch (deterministic).
 #include <cuda.h>
 
 #include <algorithm>
@@ -38,18 +49,28 @@ namespace {
 
 using namespace sm100;
 
-constexpr int KS = 5;        // slices per operand
+constexpr int KS = 5;        // slices per operand of the sweep's update
+constexpr int KSF = 7;       // slices per operand of the factorisation's products
 constexpr int SBETA = 7;     // bits per slice
-constexpr int IBM = 128;     // later columns of W per tile (UMMA M: the U slices)
-constexpr int IBN = 48;      // rows of W per tile (UMMA N: the Err slices)
+constexpr int IBM = 128;     // columns of C per tile (UMMA M: the column operand's slices)
 constexpr int IBK = 64;      // K (bytes = int8 elements) per stage: one 64-byte swizzle row
 constexpr int ISTAGES = 2;
-constexpr int IA_BYTES = KS * IBM * IBK;  // 40 KiB: U slices (UMMA A)
-constexpr int IB_BYTES = KS * IBN * IBK;  // 15 KiB: Err slices (UMMA B)
-constexpr int ISTAGE_BYTES = IA_BYTES + IB_BYTES;
 constexpr int ITHREADS = 320;
-constexpr int ISMEM = ISTAGES * ISTAGE_BYTES + 1024 + 256;
 constexpr uint32_t IWAIT = 1u << 24;
+
+// Tile shape of one kernel instance: NS slices, BN rows of C per tile (UMMA N), NBUF TMEM
+// accumulator buffers, CR rows per epilogue chunk.
+template <int NS, int BN, int NBUF>
+struct I8Shape {
+  static constexpr int A_BYTES = NS * IBM * IBK;  // column operand slices (UMMA A)
+  static constexpr int B_BYTES = NS * BN * IBK;   // row operand slices (UMMA B)
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int SMEM = ISTAGES * STAGE + 1024 + 256;
+  static_assert(NBUF * NS * BN <= 512, "accumulators exceed the tensor memory");
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N");
+};
+using SweepShape = I8Shape<KS, 48, 2>;
+using FactorShape = I8Shape<KSF, 64, 1>;
 
 __device__ int g_i8_status = 0;
 
@@ -62,8 +83,9 @@ __device__ __forceinline__ double pow2(int e) {
 __device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
 
 // ------------------------------------------------------------------ splitting
-// One warp per row of A (rows of Err[:, block], K = block width): the row exponent, then
-// KS slices of every element.  S is [KS][R][KP] (k contiguous, zero padded to KP).
+// One warp per row of A (K = the row's length): the row exponent, then NS slices of every
+// element.  S is [NS][R][KP] (k contiguous, zero padded to KP).
+template <int NS>
 __global__ void split_rows_kernel(const double* __restrict__ X, int64_t ldx, int64_t R, int64_t K, int64_t KP,
                                   int8_t* __restrict__ S, int* __restrict__ e) {
   const int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
@@ -77,7 +99,7 @@ __global__ void split_rows_kernel(const double* __restrict__ X, int64_t ldx, int
   for (int64_t k = lane; k < KP; k += 32) {
     double v = k < K ? ldexp(X[r * ldx + k], -ex) : 0.0;  // |v| < 1
 #pragma unroll
-    for (int p = 0; p < KS; ++p) {
+    for (int p = 0; p < NS; ++p) {
       v *= 128.0;
       const double sl = fmin(fmax(rint(v), -127.0), 127.0);  // nearest, |v - sl| <= 1
       v -= sl;
@@ -86,14 +108,15 @@ __global__ void split_rows_kernel(const double* __restrict__ X, int64_t ldx, int
   }
 }
 
-// Columns of B = U[block, later] (row-major, ldy): 32 columns per CTA, the column exponent,
-// then the slices transposed through shared memory into S [KS][N][KP] (k contiguous).
+// Columns of B (row-major, ldy): 32 columns per CTA, the column exponent, then the slices
+// transposed through shared memory into S [NS][N][KP] (k contiguous).
+template <int NS>
 __global__ void __launch_bounds__(256) split_cols_kernel(const double* __restrict__ Y, int64_t ldy, int64_t K,
                                                          int64_t N, int64_t KP, int8_t* __restrict__ S,
                                                          int* __restrict__ e) {
   __shared__ double mx[8][32];
   __shared__ int exs[32];
-  __shared__ int8_t tile[KS][32][33];
+  __shared__ int8_t tile[NS][32][33];
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
   const int64_t n = static_cast<int64_t>(blockIdx.x) * 32 + tx;
   double m = 0.0;
@@ -114,7 +137,7 @@ __global__ void __launch_bounds__(256) split_cols_kernel(const double* __restric
       const int64_t k = k0 + kk;
       double v = (n < N && k < K) ? ldexp(Y[k * ldy + n], -exs[tx]) : 0.0;
 #pragma unroll
-      for (int p = 0; p < KS; ++p) {
+      for (int p = 0; p < NS; ++p) {
         v *= 128.0;
         const double sl = fmin(fmax(rint(v), -127.0), 127.0);
         v -= sl;
@@ -125,21 +148,29 @@ __global__ void __launch_bounds__(256) split_cols_kernel(const double* __restric
     for (int cc = ty; cc < 32; cc += 8) {
       const int64_t nn = static_cast<int64_t>(blockIdx.x) * 32 + cc;
       if (nn < N)
-        for (int p = 0; p < KS; ++p) S[(static_cast<int64_t>(p) * N + nn) * KP + k0 + tx] = tile[p][cc][tx];
+        for (int p = 0; p < NS; ++p) S[(static_cast<int64_t>(p) * N + nn) * KP + k0 + tx] = tile[p][cc][tx];
     }
     __syncthreads();
   }
 }
 
 // ------------------------------------------------------------------ tcgen05 kind::i8 GEMM
-// 32 lanes x 16 consecutive 32-bit columns, the wait in the same statement.
-__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, int (&v)[16]) {
+// 32 lanes x 16 (or 8) consecutive 32-bit columns, the wait in the same statement.
+__device__ __forceinline__ void tmem_ld_32x32b(uint32_t taddr, int (&v)[16]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
       "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
       "tcgen05.wait::ld.sync.aligned;"
       : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
         "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld_32x32b(uint32_t taddr, int (&v)[8]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
       : "r"(taddr)
       : "memory");
 }
@@ -173,6 +204,15 @@ __host__ __device__ constexpr uint32_t i8_idesc(int M, int N) {
          ((static_cast<uint32_t>(M) >> 4) << 24);
 }
 
+// K ranges of a tile (in steps of IBK) when one operand is triangular; the skipped steps
+// multiply exact zeros.
+enum KRange : int {
+  kFullK = 0,     // every step
+  kFromCol = 1,   // column operand zero for k < column (B[k, c] = U[c, k], U upper)
+  kToCol = 2,     // column operand zero for k > column (B[k, c] = U[k, c], U upper)
+  kFromRow = 3,   // row operand zero for k < row (A[r, k] = U[r, k], U upper)
+};
+
 struct I8Args {
   int M, N, KP;               // rows, columns, padded K
   int a_rows, b_cols;         // slice strides (rows of SA per slice, columns of SB per slice)
@@ -182,13 +222,39 @@ struct I8Args {
   double* C;                  // C[r, c] for c in [0, N): C + r * ldc + c
   int64_t ldc;
   int mt, nt;
+  int krange;                 // KRange
+  int upper;                  // skip tiles strictly below the diagonal (square C, col0 == 0)
 };
 
+template <int BN>
+struct TileOf {
+  int c0, r0, kb, ke;  // first column and row, K step range [kb, ke)
+  bool skip;
+};
+
+template <int BN>
+__device__ __forceinline__ TileOf<BN> tile_of(const I8Args& a, int u) {
+  TileOf<BN> t;
+  t.c0 = (u / a.mt) * IBM;
+  t.r0 = (u % a.mt) * BN;
+  const int nk = a.KP / IBK;
+  t.kb = 0;
+  t.ke = nk;
+  if (a.krange == kFromCol) t.kb = t.c0 / IBK;
+  if (a.krange == kToCol) t.ke = min(nk, (t.c0 + IBM + IBK - 1) / IBK);
+  if (a.krange == kFromRow) t.kb = t.r0 / IBK;
+  t.kb = min(t.kb, nk - 1);  // at least one step (of zeros at worst) initialises the accumulators
+  t.skip = a.upper && t.c0 + IBM <= t.r0;
+  return t;
+}
+
+template <int NS, int BN, int NBUF, int CR>
 __global__ void __maxnreg__(160)
     i8_gemm_kernel(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb, I8Args a) {
+  using Sh = I8Shape<NS, BN, NBUF>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + ISTAGES * ISTAGE_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + ISTAGES * Sh::STAGE);
   uint64_t* empty = full + ISTAGES;
   uint64_t* accf = empty + ISTAGES;
   uint64_t* acce = accf + 2;
@@ -198,7 +264,6 @@ __global__ void __maxnreg__(160)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = static_cast<int>(gridDim.x);
   const int units = a.mt * a.nt;
-  const int nk = a.KP / IBK;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < ISTAGES; ++s) {
@@ -224,25 +289,26 @@ __global__ void __maxnreg__(160)
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer: all KS slices of A and B for one 128-wide K step
+      // ---------------- TMA producer: all NS slices of A and B for one 64-wide K step
       tma_prefetch_desc(&ta);
       tma_prefetch_desc(&tb);
       int stage = 0, issued = 0;
       uint32_t ph = 0;
       for (int u = blockIdx.x; u < units && ok; u += G) {
-        const int c0 = a.col0 + (u / a.mt) * IBM, r0 = (u % a.mt) * IBN;
-        for (int ks = 0; ks < nk; ++ks) {
+        const TileOf<BN> t = tile_of<BN>(a, u);
+        if (t.skip) continue;
+        for (int ks = t.kb; ks < t.ke; ++ks) {
           if (!mbar_wait(&empty[stage], ph ^ 1u, IWAIT)) {
             ok = false;
             break;
           }
-          uint8_t* sa = smem + stage * ISTAGE_BYTES;
-          uint8_t* sb = sa + IA_BYTES;
-          mbar_arrive_expect_tx(&full[stage], ISTAGE_BYTES);
+          uint8_t* sa = smem + stage * Sh::STAGE;
+          uint8_t* sb = sa + Sh::A_BYTES;
+          mbar_arrive_expect_tx(&full[stage], Sh::STAGE);
 #pragma unroll
-          for (int p = 0; p < KS; ++p) {
-            tma_load_2d(sa + p * IBM * IBK, &tb, &full[stage], ks * IBK, p * a.b_cols + c0);
-            tma_load_2d(sb + p * IBN * IBK, &ta, &full[stage], ks * IBK, p * a.a_rows + r0);
+          for (int p = 0; p < NS; ++p) {
+            tma_load_2d(sa + p * IBM * IBK, &tb, &full[stage], ks * IBK, p * a.b_cols + a.col0 + t.c0);
+            tma_load_2d(sb + p * BN * IBK, &ta, &full[stage], ks * IBK, p * a.a_rows + t.r0);
           }
           ++issued;
           if (++stage == ISTAGES) {
@@ -263,38 +329,42 @@ __global__ void __maxnreg__(160)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      // ---------------- UMMA issuer: 15 slice pairs (p + q <= 4) per 32-wide K substep
-      constexpr uint32_t idesc = i8_idesc(IBM, IBN);
+      // ---------------- UMMA issuer: the slice pairs p + q < NS per 32-wide K substep
+      constexpr uint32_t idesc = i8_idesc(IBM, BN);
       int stage = 0, cg = 0;
       uint32_t ph = 0;
-      for (int u = blockIdx.x; u < units && ok; u += G, ++cg) {
-        const int b = cg & 1;
-        if (!mbar_wait(&acce[b], ((cg >> 1) & 1) ^ 1u, IWAIT)) {
+      for (int u = blockIdx.x; u < units && ok; u += G) {
+        const TileOf<BN> t = tile_of<BN>(a, u);
+        if (t.skip) continue;
+        const int b = cg % NBUF;
+        const uint32_t epar = static_cast<uint32_t>((cg / NBUF) & 1);
+        ++cg;
+        if (!mbar_wait(&acce[b], epar ^ 1u, IWAIT)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t dbase = tmem + static_cast<uint32_t>(b * KS * IBN);
-        for (int ks = 0; ks < nk; ++ks) {
+        const uint32_t dbase = tmem + static_cast<uint32_t>(b * NS * BN);
+        for (int ks = t.kb; ks < t.ke; ++ks) {
           if (!mbar_wait(&full[stage], ph, IWAIT)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + stage * ISTAGE_BYTES);
-          const uint32_t sb = sa + IA_BYTES;
+          const uint32_t sa = smem_u32(smem + stage * Sh::STAGE);
+          const uint32_t sb = sa + Sh::A_BYTES;
 #pragma unroll
           for (int k = 0; k < IBK / 32; ++k) {
 #pragma unroll
-            for (int p = 0; p < KS; ++p)
+            for (int p = 0; p < NS; ++p)
 #pragma unroll
-              for (int q = 0; q < KS - p; ++q) {
+              for (int q = 0; q < NS - p; ++q) {
                 const uint64_t ad = desc_sw64(sa + p * IBM * IBK + k * 32);
-                const uint64_t bd = desc_sw64(sb + q * IBN * IBK + k * 32);
+                const uint64_t bd = desc_sw64(sb + q * BN * IBK + k * 32);
                 // pairs go p-major, so (0, s) is the first product into accumulator s: it
                 // overwrites the accumulator's previous tile
-                const bool first = ks == 0 && k == 0 && p == 0;
-                umma_i8(dbase + static_cast<uint32_t>((p + q) * IBN), ad, bd, idesc, first ? 0u : 1u);
+                const bool first = ks == t.kb && k == 0 && p == 0;
+                umma_i8(dbase + static_cast<uint32_t>((p + q) * BN), ad, bd, idesc, first ? 0u : 1u);
               }
           }
           umma_commit(&empty[stage]);
@@ -312,58 +382,71 @@ __global__ void __maxnreg__(160)
   } else {
     // ---------------- epilogue: C[r, n] -= 2^(ea_r + eb_n - 14) sum_s acc_s 2^(-7 s).  A thread
     // owns one column n (its TMEM lane); the 4 warps of each lane quarter are split over the
-    // tile's 48 rows in chunks of 16 (warps 2..5 and 6..9 take chunks 0, 2 and 1); for each
-    // row the warp's 32 lanes update 32 consecutive columns (coalesced).  The 16 loads of W are
-    // issued together before any use, and the rows of this CTA's next tile are prefetched into
-    // L2 while the current one is updated.
+    // tile's BN rows in chunks of CR (warps 2..5 take the even chunks, 6..9 the odd ones); for
+    // each row the warp's 32 lanes update 32 consecutive columns (coalesced).  The CR loads of
+    // C are issued together before any use, and the rows of this CTA's next tile are
+    // prefetched into L2 while the current one is updated.
     const int quad = warp & 3;
     const int half = (warp - 2) >> 2;
     const int et = threadIdx.x - 64;  // 0..255 over the epilogue warps
-    // L2 prefetch of the W lines (48 rows x 1 KiB) of tile u: 384 lines of 128 bytes
+    // L2 prefetch of the C lines (BN rows x 1 KiB) of tile u: 128-byte lines
     auto prefetch_tile = [&](int u) {
-      if (u >= units) return;
-      const int cb = (u / a.mt) * IBM, rb = (u % a.mt) * IBN;
-      for (int l = et; l < IBN * (IBM / 16); l += 256) {
-        const int r = rb + l / (IBM / 16), cc = cb + (l % (IBM / 16)) * 16;
-        if (r < a.M && cc < a.N) prefetch_l2(a.C + static_cast<int64_t>(r) * a.ldc + cc);
+      for (; u < units; u += G) {
+        const TileOf<BN> t = tile_of<BN>(a, u);
+        if (t.skip) continue;
+        for (int l = et; l < BN * (IBM / 16); l += 256) {
+          const int r = t.r0 + l / (IBM / 16), cc = t.c0 + (l % (IBM / 16)) * 16;
+          if (r < a.M && cc < a.N) prefetch_l2(a.C + static_cast<int64_t>(r) * a.ldc + cc);
+        }
+        return;
       }
     };
     prefetch_tile(blockIdx.x);
     int cg = 0;
-    for (int u = blockIdx.x; u < units; u += G, ++cg) {
-      const int b = cg & 1;
-      if (!mbar_wait(&accf[b], (cg >> 1) & 1, IWAIT)) {
+    for (int u = blockIdx.x; u < units; u += G) {
+      const TileOf<BN> t = tile_of<BN>(a, u);
+      if (t.skip) continue;
+      const int b = cg % NBUF;
+      const uint32_t fpar = static_cast<uint32_t>((cg / NBUF) & 1);
+      ++cg;
+      if (!mbar_wait(&accf[b], fpar, IWAIT)) {
         ok = false;
         break;
       }
       tc_fence_after();
       prefetch_tile(u + G);
-      const int c = (u / a.mt) * IBM + quad * 32 + lane;  // column within this launch
+      const int c = t.c0 + quad * 32 + lane;  // column within this launch
       const bool cin = c < a.N;
-      // 2^(eb_n - 14 - 28): the column's share of the scale, with the 2^-28 that turns the
-      // integer recombination below into sum_s acc_s 2^(-7 s)
-      const int ec = cin ? a.eb[a.col0 + c] - 2 * SBETA - (KS - 1) * SBETA : 0;
-      for (int chunk = half; chunk < IBN / 16; chunk += 2) {
-        const int r0 = (u % a.mt) * IBN + chunk * 16;
-        int acc[KS][16];
+      // The accumulators recombine exactly in 64-bit integers: hi = sum_{s<4} acc_s 2^(7(3-s))
+      // (below 2^53), and for NS > 4 lo = sum_{s>=4} acc_s 2^(7(NS-1-s)).  The value
+      // sum_s acc_s 2^(-7s) is 2^-21 (hi + lo 2^(-7(NS-4))), formed with one rounding.
+      const int ec = cin ? a.eb[a.col0 + c] - 2 * SBETA - 3 * SBETA : 0;
+      for (int chunk = half; chunk < BN / CR; chunk += 2) {
+        const int r0 = t.r0 + chunk * CR;
+        int acc[NS][CR];
 #pragma unroll
-        for (int s = 0; s < KS; ++s)
-          tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(quad * 32) << 16) +
-                                 static_cast<uint32_t>(b * KS * IBN + s * IBN + chunk * 16),
-                             acc[s]);
-        double cv[16];
+        for (int s = 0; s < NS; ++s)
+          tmem_ld_32x32b(tmem + (static_cast<uint32_t>(quad * 32) << 16) +
+                             static_cast<uint32_t>(b * NS * BN + s * BN + chunk * CR),
+                         acc[s]);
+        double cv[CR];
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
+        for (int j = 0; j < CR; ++j)
           cv[j] = (cin && r0 + j < a.M) ? a.C[static_cast<int64_t>(r0 + j) * a.ldc + c] : 0.0;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          // sum_s acc_s 2^(7 (KS-1-s)) exactly in 64-bit integers (|acc_s| < 2^31, so the sum
-          // stays below 2^60), then one rounding to fp64 and an exact power-of-two scale
-          long long v = acc[0][j];
+        for (int j = 0; j < CR; ++j) {
+          long long hi = acc[0][j];
 #pragma unroll
-          for (int s = 1; s < KS; ++s) v = v * (1ll << SBETA) + acc[s][j];
+          for (int s = 1; s < 4; ++s) hi = hi * (1ll << SBETA) + acc[s][j];
+          double v = static_cast<double>(hi);
+          if constexpr (NS > 4) {
+            long long lo = acc[4][j];
+#pragma unroll
+            for (int s = 5; s < NS; ++s) lo = lo * (1ll << SBETA) + acc[s][j];
+            v = fma(static_cast<double>(lo), pow2(-SBETA * (NS - 4)), v);
+          }
           if (cin && r0 + j < a.M)
-            a.C[static_cast<int64_t>(r0 + j) * a.ldc + c] = cv[j] - static_cast<double>(v) * pow2(ec + a.ea[r0 + j]);
+            a.C[static_cast<int64_t>(r0 + j) * a.ldc + c] = cv[j] - v * pow2(ec + a.ea[r0 + j]);
         }
       }
       tc_fence_before();
@@ -411,40 +494,36 @@ int slice_map(CUtensorMap* tm, const int8_t* base, int64_t rows, int64_t KP, int
   return r == CUDA_SUCCESS ? GPTQ_OK : GPTQ_ERR_CUDA;
 }
 
-}  // namespace
-
-int i8_slices() { return KS; }
-int64_t i8_padded_k(int64_t K) { return ((K + IBK - 1) / IBK) * IBK; }
-
-int i8_split_rows(cudaStream_t s, const double* X, int64_t ldx, int64_t R, int64_t K, int64_t KP, int8_t* S, int* e) {
+template <int NS>
+int split_rows_any(cudaStream_t s, const double* X, int64_t ldx, int64_t R, int64_t K, int64_t KP, int8_t* S, int* e) {
   if (R <= 0) return GPTQ_OK;
-  split_rows_kernel<<<static_cast<unsigned>((R + 7) / 8), 256, 0, s>>>(X, ldx, R, K, KP, S, e);
+  split_rows_kernel<NS><<<static_cast<unsigned>((R + 7) / 8), 256, 0, s>>>(X, ldx, R, K, KP, S, e);
   return after_launch();
 }
 
-int i8_split_cols(cudaStream_t s, const double* Y, int64_t ldy, int64_t K, int64_t N, int64_t KP, int8_t* S, int* e) {
+template <int NS>
+int split_cols_any(cudaStream_t s, const double* Y, int64_t ldy, int64_t K, int64_t N, int64_t KP, int8_t* S, int* e) {
   if (N <= 0) return GPTQ_OK;
-  split_cols_kernel<<<static_cast<unsigned>((N + 31) / 32), 256, 0, s>>>(Y, ldy, K, N, KP, S, e);
+  split_cols_kernel<NS><<<static_cast<unsigned>((N + 31) / 32), 256, 0, s>>>(Y, ldy, K, N, KP, S, e);
   return after_launch();
 }
 
-// C[r, c] -= (A B)[r, col0 + c] for r < M, c < N, from the slices of i8_split_rows (SA,
-// a_rows rows per slice, exponents ea) and i8_split_cols (SB, b_cols columns per slice,
-// exponents eb), K padded to KP.  The persistent grid has at most max_ctas CTAs (0: one per
-// SM): a CTA takes most of an SM's shared memory, so a launch that runs beside other
-// kernels leaves them SMs of their own.
-int i8_gemm_sub(cudaStream_t s, int64_t M, int64_t N, int64_t KP, const int8_t* SA, int64_t a_rows, const int* ea,
-                const int8_t* SB, int64_t b_cols, const int* eb, int64_t col0, double* C, int64_t ldc,
-                int max_ctas) {
+template <int NS, int BN, int NBUF, int CR>
+int gemm_any(cudaStream_t s, int64_t M, int64_t N, int64_t KP, const int8_t* SA, int64_t a_rows, const int* ea,
+             const int8_t* SB, int64_t b_cols, const int* eb, int64_t col0, double* C, int64_t ldc, int max_ctas,
+             int krange, int upper) {
+  using Sh = I8Shape<NS, BN, NBUF>;
   if (M <= 0 || N <= 0) return GPTQ_OK;
   // Rows past a slice's end (a tile reaching beyond M) load the next slice's first rows, or
   // zeros past the last slice; they only reach accumulator rows (columns) >= M (N), which
   // the epilogue never writes.
   if (KP % IBK != 0 || KP > 16384 || M > a_rows || col0 + N > b_cols) return GPTQ_ERR_UNSUPPORTED;
-  GPTQ_TRY(ensure_smem_limit(reinterpret_cast<const void*>(i8_gemm_kernel), ISMEM));
+  if (upper && (col0 != 0 || M != N)) return GPTQ_ERR_UNSUPPORTED;
+  auto kern = i8_gemm_kernel<NS, BN, NBUF, CR>;
+  GPTQ_TRY(ensure_smem_limit(reinterpret_cast<const void*>(kern), Sh::SMEM));
   CUtensorMap ta, tb;
-  GPTQ_TRY(slice_map(&ta, SA, KS * a_rows, KP, IBN));
-  GPTQ_TRY(slice_map(&tb, SB, KS * b_cols, KP, IBM));
+  GPTQ_TRY(slice_map(&ta, SA, NS * a_rows, KP, BN));
+  GPTQ_TRY(slice_map(&tb, SB, NS * b_cols, KP, IBM));
   I8Args a;
   a.M = static_cast<int>(M);
   a.N = static_cast<int>(N);
@@ -456,12 +535,55 @@ int i8_gemm_sub(cudaStream_t s, int64_t M, int64_t N, int64_t KP, const int8_t* 
   a.col0 = static_cast<int>(col0);
   a.C = C;
   a.ldc = ldc;
-  a.mt = static_cast<int>((M + IBN - 1) / IBN);  // row tiles of 64
+  a.mt = static_cast<int>((M + BN - 1) / BN);    // row tiles
   a.nt = static_cast<int>((N + IBM - 1) / IBM);  // column tiles of 128
+  a.krange = krange;
+  a.upper = upper;
   const int cap = max_ctas > 0 ? std::min(max_ctas, num_sms()) : num_sms();
   const int grid = static_cast<int>(std::min<int64_t>(cap, static_cast<int64_t>(a.mt) * a.nt));
-  i8_gemm_kernel<<<grid, ITHREADS, ISMEM, s>>>(ta, tb, a);
+  kern<<<grid, ITHREADS, Sh::SMEM, s>>>(ta, tb, a);
   return after_launch();
+}
+
+}  // namespace
+
+int i8_slices() { return KS; }
+int i8f_slices() { return KSF; }
+int64_t i8_padded_k(int64_t K) { return ((K + IBK - 1) / IBK) * IBK; }
+
+int i8_split_rows(cudaStream_t s, const double* X, int64_t ldx, int64_t R, int64_t K, int64_t KP, int8_t* S, int* e) {
+  return split_rows_any<KS>(s, X, ldx, R, K, KP, S, e);
+}
+int i8_split_cols(cudaStream_t s, const double* Y, int64_t ldy, int64_t K, int64_t N, int64_t KP, int8_t* S, int* e) {
+  return split_cols_any<KS>(s, Y, ldy, K, N, KP, S, e);
+}
+int i8f_split_rows(cudaStream_t s, const double* X, int64_t ldx, int64_t R, int64_t K, int64_t KP, int8_t* S, int* e) {
+  return split_rows_any<KSF>(s, X, ldx, R, K, KP, S, e);
+}
+int i8f_split_cols(cudaStream_t s, const double* Y, int64_t ldy, int64_t K, int64_t N, int64_t KP, int8_t* S,
+                   int* e) {
+  return split_cols_any<KSF>(s, Y, ldy, K, N, KP, S, e);
+}
+
+// C[r, c] -= (A B)[r, col0 + c] for r < M, c < N, from the slices of i8_split_rows (SA,
+// a_rows rows per slice, exponents ea) and i8_split_cols (SB, b_cols columns per slice,
+// exponents eb), K padded to KP.  The persistent grid has at most max_ctas CTAs (0: one per
+// SM): a CTA takes most of an SM's shared memory, so a launch that runs beside other
+// kernels leaves them SMs of their own.
+int i8_gemm_sub(cudaStream_t s, int64_t M, int64_t N, int64_t KP, const int8_t* SA, int64_t a_rows, const int* ea,
+                const int8_t* SB, int64_t b_cols, const int* eb, int64_t col0, double* C, int64_t ldc,
+                int max_ctas) {
+  return gemm_any<KS, 48, 2, 16>(s, M, N, KP, SA, a_rows, ea, SB, b_cols, eb, col0, C, ldc, max_ctas, kFullK, 0);
+}
+
+// The factorisation's products: C[r, c] -= (A B)[r, c] from seven-slice operands (i8f_split_*),
+// with the K steps a triangular operand makes zero skipped (krange: 0 none, 1 B[k, c] = 0 for
+// k < c, 2 B[k, c] = 0 for k > c, 3 A[r, k] = 0 for k < r) and, with upper, only the tiles
+// that reach the diagonal or above (square C).
+int i8f_gemm_sub(cudaStream_t s, int64_t M, int64_t N, int64_t KP, const int8_t* SA, int64_t a_rows, const int* ea,
+                 const int8_t* SB, int64_t b_cols, const int* eb, double* C, int64_t ldc, int krange, int upper) {
+  if (krange < kFullK || krange > kFromRow) return GPTQ_ERR_INVALID_ARG;
+  return gemm_any<KSF, 64, 1, 8>(s, M, N, KP, SA, a_rows, ea, SB, b_cols, eb, 0, C, ldc, 0, krange, upper);
 }
 
 int i8_device_status(int clear) {
