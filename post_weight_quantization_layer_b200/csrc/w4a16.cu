@@ -302,93 +302,206 @@ __global__ void __launch_bounds__(GTHREADS, 1)
 constexpr int GV_THREADS = 256;  // 8 warps; a lane owns 4 consecutive outputs
 constexpr int GV_N = 128;        // outputs per CTA
 constexpr int GV_MAXM = 4;
+constexpr int GV_ROWS = 4;       // word rows of one warp in flight
 
+// Packed fp32 pairs (the f32x2 arithmetic of sm_100).
+__device__ __forceinline__ unsigned long long f2_bits(float2 v) { return *reinterpret_cast<unsigned long long*>(&v); }
+__device__ __forceinline__ float2 bits_f2(unsigned long long b) { return *reinterpret_cast<float2*>(&b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
+  return bits_f2(d);
+}
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  unsigned long long d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return bits_f2(d);
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return bits_f2(d);
+}
+
+// Group parameters of one output in the form the paired dequantization wants, and the
+// pair itself: codes i and i + FPW/2 of a word (the same bit offset in its two 16-bit
+// halves), both returned as round16(s * (q - z)) in a float2.
+//  * float16: 0x6400 | q is the half 1024 + q (exact for q < 1024); subtracting 1024 + z
+//    leaves q - z exactly, and one half multiply by s rounds the exact product once, to
+//    nearest even: round16(s * (q - z)), two codes per instruction.
+//  * bfloat16: the same in fp32 (0x4B000000 | q is 2^23 + q): q - z and s * (q - z) are
+//    exact in fp32 (a 19-bit product), then one rounding to bfloat16.
+template <typename T>
+struct PairDeq;
+template <>
+struct PairDeq<__half> {
+  __half2 s2, zb2;
+  __device__ __forceinline__ void set(float s, int z) {
+    s2 = __float2half2_rn(s);  // s is a float16 value: exact
+    zb2 = __float2half2_rn(1024.f + static_cast<float>(z));
+  }
+  template <int BITS>
+  __device__ __forceinline__ float2 pair(uint32_t w, int i) const {
+    constexpr uint32_t m = (1u << BITS) - 1u;
+    const uint32_t h = ((w >> (i * BITS)) & ((m << 16) | m)) | 0x64006400u;
+    const __half2 v = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&h), zb2), s2);
+    return __half22float2(v);
+  }
+};
+template <>
+struct PairDeq<__nv_bfloat16> {
+  float2 s2, zb2;
+  __device__ __forceinline__ void set(float s, int z) {
+    s2 = make_float2(s, s);
+    zb2 = make_float2(8388608.f + static_cast<float>(z), 8388608.f + static_cast<float>(z));
+  }
+  template <int BITS>
+  __device__ __forceinline__ float2 pair(uint32_t w, int i) const {
+    constexpr uint32_t m = (1u << BITS) - 1u;
+    const uint32_t lo = (w >> (i * BITS)) & m, hi = (w >> (i * BITS + 16)) & m;
+    const float2 q = make_float2(__uint_as_float(0x4B000000u | lo), __uint_as_float(0x4B000000u | hi));
+    const __nv_bfloat162 b = __float22bfloat162_rn(mul2(sub2(q, zb2), s2));
+    return __bfloat1622float2(b);
+  }
+};
+
+// One CTA: 128 outputs x one K chunk.  The chunk's activations are staged in shared memory
+// as pairs (x[k], x[k + FPW/2]) matching the paired codes, and every word row is marked
+// with its group when all its FPW codes share one (always for checkpoints whose g_idx runs
+// in order), else -1.  Rows of one group take the paired path with the group parameters
+// loaded once per group; mixed rows (act-order checkpoints) take a per-code path with a
+// group lookup for every code.  Each warp keeps GV_ROWS word rows in flight (16-byte loads,
+// a warp reads 512 contiguous bytes of a row); fp32 products are accumulated in pairs.
 template <int BITS, typename T, int MM>
-__global__ void __launch_bounds__(GV_THREADS) gemv_kernel(const T* __restrict__ X, int M, int64_t K,
+__global__ void __launch_bounds__(GV_THREADS, 2) gemv_kernel(const T* __restrict__ X, int M, int64_t K,
                                                           const int32_t* __restrict__ qweight,
                                                           const int32_t* __restrict__ qzeros,
                                                           const __half* __restrict__ scales,
                                                           const int32_t* __restrict__ g_idx, int G, int64_t N,
                                                           int kchunk, float* __restrict__ partial) {
   constexpr int FPW = 32 / BITS;
+  constexpr int HP = FPW / 2;  // code pairs per word
   constexpr uint32_t MASK = (1u << BITS) - 1u;
   extern __shared__ __align__(16) float gsm[];
-  float* xs = gsm;                                     // [GV_MAXM][kchunk]
-  int* gs = reinterpret_cast<int*>(xs + GV_MAXM * kchunk);  // [kchunk]
-  float* red = reinterpret_cast<float*>(gs + kchunk);  // [8][GV_MAXM][GV_N]
+  float2* xs = reinterpret_cast<float2*>(gsm);            // [MM][kchunk / 2] pairs
+  int* gs = reinterpret_cast<int*>(gsm + MM * kchunk);     // [kchunk] group of each k
+  int* rg = gs + kchunk;                                   // [kchunk / FPW] group of each row
+  float* red = reinterpret_cast<float*>(rg + kchunk / 4);  // [8][MM][GV_N] (FPW >= 4)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t klo = static_cast<int64_t>(blockIdx.y) * kchunk;
   const int kn = static_cast<int>(min(static_cast<int64_t>(kchunk), K - klo));
+  const int rows = kn / FPW;  // kchunk and K are multiples of FPW
   for (int e = tid; e < kn; e += GV_THREADS) {
     gs[e] = clamp_group(__ldg(g_idx + klo + e), G);
+    // k = r*FPW + f sits in pair slot r*HP + (f mod HP), component f / HP
+    const int r = e / FPW, f = e % FPW;
+    float* slot = reinterpret_cast<float*>(xs + r * HP + (f % HP)) + (f / HP);
 #pragma unroll
-    for (int m = 0; m < MM; ++m) xs[m * kchunk + e] = to_f32<T>(X[m * K + klo + e]);
+    for (int m = 0; m < MM; ++m) slot[m * kchunk] = to_f32<T>(X[m * K + klo + e]);
+  }
+  __syncthreads();
+  for (int r = tid; r < rows; r += GV_THREADS) {
+    const int g0 = gs[r * FPW];
+    bool same = true;
+#pragma unroll
+    for (int f = 1; f < FPW; ++f) same = same && gs[r * FPW + f] == g0;
+    rg[r] = same ? g0 : -1;
   }
   __syncthreads();
   const int64_t n = static_cast<int64_t>(blockIdx.x) * GV_N + lane * 4;
-  float acc[MM][4];
+  float2 acc[MM][4];
 #pragma unroll
   for (int m = 0; m < MM; ++m)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[m][j] = 0.f;
+    for (int j = 0; j < 4; ++j) acc[m][j] = make_float2(0.f, 0.f);
   if (n < N) {
     const int64_t zw = N * BITS / 32;
     const int zshift = static_cast<int>((n * BITS) % 32);
-    const int rows = kn / FPW;  // kchunk and K are multiples of FPW
     int gcur = -1;
-    float s[4];
-    int z[4];
-    // one word row of 4 outputs: its FPW codes each, with the group parameters of each code's k
+    PairDeq<T> pd[4];
+    float sc[4];
+    int zc[4];
+    auto load_group = [&](int g) {
+      gcur = g;
+      const uint2 s4 = __ldg(reinterpret_cast<const uint2*>(scales + static_cast<int64_t>(g) * N + n));
+      const __half2 s01 = *reinterpret_cast<const __half2*>(&s4.x);
+      const __half2 s23 = *reinterpret_cast<const __half2*>(&s4.y);
+      sc[0] = __low2float(s01);
+      sc[1] = __high2float(s01);
+      sc[2] = __low2float(s23);
+      sc[3] = __high2float(s23);
+      const uint32_t zword = static_cast<uint32_t>(__ldg(qzeros + static_cast<int64_t>(g) * zw + (n * BITS) / 32));
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        zc[j] = static_cast<int>((zword >> (zshift + j * BITS)) & MASK);
+        pd[j].set(sc[j], zc[j]);
+      }
+    };
     auto row_math = [&](int r, const int4 w4) {
       const uint32_t wv[4] = {static_cast<uint32_t>(w4.x), static_cast<uint32_t>(w4.y), static_cast<uint32_t>(w4.z),
                               static_cast<uint32_t>(w4.w)};
+      const int g = rg[r];
+      if (g >= 0) {
+        if (g != gcur) load_group(g);
 #pragma unroll
-      for (int f = 0; f < FPW; ++f) {
-        const int kl = r * FPW + f;
-        const int g = gs[kl];
-        if (g != gcur) {
-          gcur = g;
-          const uint2 s4 = __ldg(reinterpret_cast<const uint2*>(scales + static_cast<int64_t>(g) * N + n));
-          const __half2 s01 = *reinterpret_cast<const __half2*>(&s4.x);
-          const __half2 s23 = *reinterpret_cast<const __half2*>(&s4.y);
-          s[0] = __low2float(s01);
-          s[1] = __high2float(s01);
-          s[2] = __low2float(s23);
-          s[3] = __high2float(s23);
-          const uint32_t zword = static_cast<uint32_t>(__ldg(qzeros + static_cast<int64_t>(g) * zw + (n * BITS) / 32));
+        for (int i = 0; i < HP; ++i) {
+          float2 xp[MM];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) z[j] = static_cast<int>((zword >> (zshift + j * BITS)) & MASK);
+          for (int m = 0; m < MM; ++m) xp[m] = xs[m * (kchunk / 2) + r * HP + i];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 w = pd[j].template pair<BITS>(wv[j], i);
+#pragma unroll
+            for (int m = 0; m < MM; ++m) acc[m][j] = fma2(xp[m], w, acc[m][j]);
+          }
         }
+      } else {
+        // mixed groups within the row: one code at a time
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float w = dq<T>(s[j], static_cast<int>((wv[j] >> (f * BITS)) & MASK), z[j]);
+        for (int f = 0; f < FPW; ++f) {
+          const int gk = gs[r * FPW + f];
+          if (gk != gcur) load_group(gk);
+          const int slot = r * HP + (f % HP);
 #pragma unroll
-          for (int m = 0; m < MM; ++m) acc[m][j] = fmaf(xs[m * kchunk + kl], w, acc[m][j]);
+          for (int j = 0; j < 4; ++j) {
+            const float w = dq<T>(sc[j], static_cast<int>((wv[j] >> (f * BITS)) & MASK), zc[j]);
+#pragma unroll
+            for (int m = 0; m < MM; ++m) {
+              const float x = reinterpret_cast<const float*>(xs + m * (kchunk / 2) + slot)[f / HP];
+              if (f / HP == 0)
+                acc[m][j].x = fmaf(x, w, acc[m][j].x);
+              else
+                acc[m][j].y = fmaf(x, w, acc[m][j].y);
+            }
+          }
         }
       }
     };
     const int64_t wbase = klo / FPW;
+    constexpr int RF = BITS == 2 ? 2 : GV_ROWS;  // 2-bit rows unpack twice the codes
     int r = warp;
-    for (; r + 8 < rows; r += 16) {  // two word rows in flight
-      const int4 wa = __ldg(reinterpret_cast<const int4*>(qweight + (wbase + r) * N + n));
-      const int4 wb = __ldg(reinterpret_cast<const int4*>(qweight + (wbase + r + 8) * N + n));
-      row_math(r, wa);
-      row_math(r + 8, wb);
+    for (; r + 8 * (RF - 1) < rows; r += 8 * RF) {
+      int4 w[RF];
+#pragma unroll
+      for (int t = 0; t < RF; ++t)
+        w[t] = __ldg(reinterpret_cast<const int4*>(qweight + (wbase + r + 8 * t) * N + n));
+#pragma unroll
+      for (int t = 0; t < RF; ++t) row_math(r + 8 * t, w[t]);
     }
-    if (r < rows) row_math(r, __ldg(reinterpret_cast<const int4*>(qweight + (wbase + r) * N + n)));
+    for (; r < rows; r += 8) row_math(r, __ldg(reinterpret_cast<const int4*>(qweight + (wbase + r) * N + n)));
   }
   // the 8 warps' partial sums of this CTA's outputs, added in a fixed order
 #pragma unroll
   for (int m = 0; m < MM; ++m)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) red[(warp * GV_MAXM + m) * GV_N + lane * 4 + j] = acc[m][j];
+    for (int j = 0; j < 4; ++j) red[(warp * MM + m) * GV_N + lane * 4 + j] = acc[m][j].x + acc[m][j].y;
   __syncthreads();
   for (int e = tid; e < MM * GV_N; e += GV_THREADS) {
     const int m = e / GV_N, c = e % GV_N;
     const int64_t nn = static_cast<int64_t>(blockIdx.x) * GV_N + c;
     if (m < M && nn < N) {
       float t = 0.f;
-      for (int w = 0; w < 8; ++w) t += red[(w * GV_MAXM + m) * GV_N + c];
+      for (int w = 0; w < 8; ++w) t += red[(w * MM + m) * GV_N + c];
       partial[(static_cast<int64_t>(blockIdx.y) * M + m) * N + nn] = t;
     }
   }
@@ -478,7 +591,7 @@ int launch_gemv(const T* X, int M, int64_t K, const int32_t* qw, const int32_t* 
   kchunk = std::min<int64_t>(kchunk, 4096);
   S = (K + kchunk - 1) / kchunk;
   if (S > 65535) return GPTQ_ERR_UNSUPPORTED;
-  const size_t smem = (GV_MAXM * kchunk + kchunk) * 4 + 8 * GV_MAXM * GV_N * 4;
+  const size_t smem = (MM * kchunk + kchunk + kchunk / 4) * 4 + 8 * MM * GV_N * 4;
   GPTQ_TRY(ensure_smem_limit(reinterpret_cast<const void*>(gemv_kernel<BITS, T, MM>), static_cast<int>(smem)));
   float* partial = nullptr;
   GPTQ_TRY(pool_alloc(reinterpret_cast<void**>(&partial), static_cast<size_t>(S) * M * N * 4, s));
