@@ -702,8 +702,10 @@ def run_qlinear(args):
     packed codes + fp16 scales + packed zero points + g_idx + X + Y) against the measured
     copy bandwidth, the dequantization (bytes = the checkpoint read + the 16-bit weight
     written) likewise, and the tensor-core GEMM (2 M N K flops) against the measured bf16
-    rate.  CUDA events on the launching stream, 3 warm-ups, the median of 20 launches;
-    weights are re-read every launch (decode shapes below L2 are reported as such)."""
+    rate.  Device time: the call's launches captured once in a CUDA graph and replayed, CUDA
+    events around each replay, 3 warm-ups, the median of 20; decode also reports the wall time
+    of one call through the Python binding (call_us, host overhead included).  Weights are
+    re-read every launch (decode shapes below L2 are reported as such)."""
     import torch
 
     import post_weight_quantization_layer_b200 as gq
@@ -715,17 +717,51 @@ def run_qlinear(args):
     stream = torch.cuda.current_stream()
 
     def timed(fn, reps=20):
+        """Device time of one fn() (median over reps), its launches replayed from a CUDA graph
+        so that the host-side cost of the Python call is not in the number."""
         for _ in range(3):
             fn()
+        torch.cuda.synchronize()
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        g = torch.cuda.CUDAGraph()
+        try:
+            with torch.cuda.stream(side), torch.cuda.graph(g, stream=side):
+                fn()
+        except RuntimeError as e:  # not capturable: time back-to-back calls instead
+            print(f"graph capture failed ({e}); timing 20 queued calls", file=sys.stderr)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                fn()
+            e1.record(stream)
+            e1.synchronize()
+            return e0.elapsed_time(e1) / reps
+        torch.cuda.synchronize()
         ts = []
         for _ in range(reps):
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            fn()
+            g.replay()
             e1.record(stream)
             e1.synchronize()
             ts.append(e0.elapsed_time(e1))
+        del g
         return statistics.median(ts)
+
+    def call_timed(fn, reps=20):
+        """Wall time of one call through the Python binding, host overhead included."""
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            t0 = time.perf_counter()
+            fn()
+            torch.cuda.synchronize()
+            ts.append(time.perf_counter() - t0)
+        return statistics.median(ts) * 1e3
 
     out = {"mode": "qlinear", "unit_decode": "GB/s", "unit_gemm": "TFLOP/s", "hbm_peak_gbs": peaks["hbm"],
            "bf16_peak_tflops": peaks["bf16"], "peaks": peaks["source"], "shapes": []}
@@ -752,15 +788,18 @@ def run_qlinear(args):
             for M in (1, 4):
                 X = torch.randn(M, n_in, device=dev).to(torch.bfloat16)
                 Y = torch.empty(M, n_out, device=dev, dtype=torch.bfloat16)
-                ms = timed(lambda: gq.quantized_linear(X, c, bits, out=Y))
+                fn = lambda: gq.quantized_linear(X, c, bits, out=Y)  # noqa: E731
+                ms = timed(fn)
                 gbs = (wbytes + M * (n_in + n_out) * 2) / (ms / 1e3) / 1e9
                 row[f"decode_m{M}{tag}"] = {"us": round(ms * 1e3, 1), "gbs": round(gbs, 1),
                                             "frac_of_hbm": round(gbs / peaks["hbm"], 3),
-                                            "l2_resident": wbytes < 100e6}
+                                            "l2_resident": wbytes < 100e6,
+                                            "call_us": round(call_timed(fn) * 1e3, 1)}
         Wd = torch.empty(n_out, n_in, dtype=torch.bfloat16, device=dev)
         ms = timed(lambda: lib().gptq_dequantize_weight(ck["qweight"].data_ptr(), ck["qzeros"].data_ptr(),
                                                          ck["scales"].data_ptr(), ck["g_idx"].data_ptr(), G, n_in,
-                                                         n_out, bits, 2, Wd.data_ptr(), stream.cuda_stream))
+                                                         n_out, bits, 2, Wd.data_ptr(),
+                                                         torch.cuda.current_stream().cuda_stream))
         gbs = (wbytes + n_in * n_out * 2) / (ms / 1e3) / 1e9
         row["dequant"] = {"us": round(ms * 1e3, 1), "gbs": round(gbs, 1), "frac_of_hbm": round(gbs / peaks["hbm"], 3)}
         for M in (2048, 16384):

@@ -40,6 +40,10 @@ cudaMemPool_t workspace_pool() {
   }
   uint64_t thr = UINT64_MAX;
   cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &thr);
+  // No reuse of a block freed on another stream through an inserted wait: concurrent calls
+  // (the sweeps of one pipelined layer on their own streams) would queue behind each other.
+  int no = 0;
+  cudaMemPoolSetAttribute(pool, cudaMemPoolReuseAllowInternalDependencies, &no);
   g_pools[dev] = pool;
   return pool;
 }
