@@ -83,74 +83,111 @@ __device__ __forceinline__ double pow2(int e) {
 __device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
 
 // ------------------------------------------------------------------ splitting
-// One warp per row of A (K = the row's length): the row exponent, then NS slices of every
-// element.  S is [NS][R][KP] (k contiguous, zero padded to KP).
+// The NS slices of v (|v| < 1), each rounded to nearest and clamped to [-127, 127]; the
+// remainder carries to the next slice.
+template <int NS>
+__device__ __forceinline__ void slices_of(double v, int8_t (&sl)[NS]) {
+#pragma unroll
+  for (int p = 0; p < NS; ++p) {
+    v *= 128.0;
+    const double r = fmin(fmax(rint(v), -127.0), 127.0);  // nearest, |v - r| <= 1
+    v -= r;
+    sl[p] = static_cast<int8_t>(r);
+  }
+}
+
+// One warp per row of A (K = the row's length): the row exponent (2^e > max |row|), then NS
+// slices of every element.  S is [NS][R][KP] (k contiguous, zero padded to KP).  A lane takes
+// 4 consecutive k and stores 4 slice bytes at once.
 template <int NS>
 __global__ void split_rows_kernel(const double* __restrict__ X, int64_t ldx, int64_t R, int64_t K, int64_t KP,
                                   int8_t* __restrict__ S, int* __restrict__ e) {
   const int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
   const int lane = threadIdx.x & 31;
   if (r >= R) return;
+  const double* x = X + r * ldx;
   double m = 0.0;
-  for (int64_t k = lane; k < K; k += 32) m = fmax(m, fabs(X[r * ldx + k]));
+  for (int64_t k = lane; k < K; k += 32) m = fmax(m, fabs(x[k]));
   for (int off = 16; off; off >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, off));
   const int ex = m > 0.0 ? ilogb(m) + 1 : 0;  // 2^ex > m
   if (lane == 0) e[r] = ex;
-  for (int64_t k = lane; k < KP; k += 32) {
-    double v = k < K ? ldexp(X[r * ldx + k], -ex) : 0.0;  // |v| < 1
+  for (int64_t k0 = 4 * lane; k0 < KP; k0 += 128) {  // KP is a multiple of 64
+    uint32_t w[NS];
 #pragma unroll
-    for (int p = 0; p < NS; ++p) {
-      v *= 128.0;
-      const double sl = fmin(fmax(rint(v), -127.0), 127.0);  // nearest, |v - sl| <= 1
-      v -= sl;
-      S[(static_cast<int64_t>(p) * R + r) * KP + k] = static_cast<int8_t>(sl);
+    for (int p = 0; p < NS; ++p) w[p] = 0;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int64_t k = k0 + t;
+      int8_t sl[NS];
+      slices_of<NS>(k < K ? ldexp(x[k], -ex) : 0.0, sl);
+#pragma unroll
+      for (int p = 0; p < NS; ++p) w[p] |= static_cast<uint32_t>(static_cast<uint8_t>(sl[p])) << (8 * t);
     }
+#pragma unroll
+    for (int p = 0; p < NS; ++p) *reinterpret_cast<uint32_t*>(S + (static_cast<int64_t>(p) * R + r) * KP + k0) = w[p];
   }
 }
 
-// Columns of B (row-major, ldy): 32 columns per CTA, the column exponent, then the slices
-// transposed through shared memory into S [NS][N][KP] (k contiguous).
-template <int NS>
-__global__ void __launch_bounds__(256) split_cols_kernel(const double* __restrict__ Y, int64_t ldy, int64_t K,
-                                                         int64_t N, int64_t KP, int8_t* __restrict__ S,
-                                                         int* __restrict__ e) {
-  __shared__ double mx[8][32];
-  __shared__ int exs[32];
-  __shared__ int8_t tile[NS][32][33];
+// Columns of B (row-major, ldy), in three steps.  col_exp_init: e[n] = -2000 (no column yet
+// seen).  col_exp_kernel: per 32 columns x 256 rows, the largest ilogb(|y|) + 1, merged into e
+// with atomicMax (the exponent of a column's maximum is the maximum of its exponents; the
+// result does not depend on the order).  An all-zero column keeps -2000, which scales its
+// (zero) slices to zero in the product.  col_slices_kernel: per 32 columns x 128 k, the
+// slices transposed through shared memory into S [NS][N][KP] (k contiguous, 128-byte rows).
+__global__ void col_exp_init_kernel(int* __restrict__ e, int64_t N) {
+  const int64_t n = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (n < N) e[n] = -2000;
+}
+
+constexpr int CE_ROWS = 256;
+__global__ void __launch_bounds__(256) col_exp_kernel(const double* __restrict__ Y, int64_t ldy, int64_t K,
+                                                      int64_t N, int* __restrict__ e) {
+  __shared__ int mx[8][32];
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
   const int64_t n = static_cast<int64_t>(blockIdx.x) * 32 + tx;
-  double m = 0.0;
+  const int64_t k0 = static_cast<int64_t>(blockIdx.y) * CE_ROWS;
+  int best = -2000;
   if (n < N)
-    for (int64_t k = ty; k < K; k += 8) m = fmax(m, fabs(Y[k * ldy + n]));
-  mx[ty][tx] = m;
+    for (int64_t k = k0 + ty; k < min(K, k0 + CE_ROWS); k += 8) {
+      const double v = fabs(Y[k * ldy + n]);
+      if (v > 0.0) best = max(best, ilogb(v) + 1);
+    }
+  mx[ty][tx] = best;
   __syncthreads();
-  if (ty == 0) {
-    double mm = 0.0;
-    for (int i = 0; i < 8; ++i) mm = fmax(mm, mx[i][tx]);
-    const int ex = mm > 0.0 ? ilogb(mm) + 1 : 0;
-    exs[tx] = ex;
-    if (n < N) e[n] = ex;
+  if (ty == 0 && n < N) {
+    for (int i = 1; i < 8; ++i) best = max(best, mx[i][tx]);
+    if (best > -2000) atomicMax(e + n, best);
+  }
+}
+
+constexpr int CS_K = 128;
+template <int NS, int KW>
+__global__ void __launch_bounds__(256) col_slices_kernel(const double* __restrict__ Y, int64_t ldy, int64_t K,
+                                                         int64_t N, int64_t KP, int64_t kbase,
+                                                         int8_t* __restrict__ S, const int* __restrict__ e) {
+  constexpr int PITCH = KW + 4;  // bytes per tile row (4-byte aligned, spreads the banks)
+  constexpr int WPR = KW / 4;    // 32-bit words per output row
+  __shared__ __align__(16) int8_t tile[NS][32][PITCH];
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int64_t n = static_cast<int64_t>(blockIdx.x) * 32 + tx;
+  const int64_t k0 = kbase + static_cast<int64_t>(blockIdx.y) * KW;
+  const int ex = n < N ? max(e[n], -1100) : 0;  // a zero column's slices are zero whatever ex
+  for (int kk = ty; kk < KW; kk += 8) {
+    const int64_t k = k0 + kk;
+    int8_t sl[NS];
+    slices_of<NS>((n < N && k < K) ? ldexp(Y[k * ldy + n], -ex) : 0.0, sl);
+#pragma unroll
+    for (int p = 0; p < NS; ++p) tile[p][tx][kk] = sl[p];
   }
   __syncthreads();
-  for (int64_t k0 = 0; k0 < KP; k0 += 32) {
-    for (int kk = ty; kk < 32; kk += 8) {
-      const int64_t k = k0 + kk;
-      double v = (n < N && k < K) ? ldexp(Y[k * ldy + n], -exs[tx]) : 0.0;
-#pragma unroll
-      for (int p = 0; p < NS; ++p) {
-        v *= 128.0;
-        const double sl = fmin(fmax(rint(v), -127.0), 127.0);
-        v -= sl;
-        tile[p][tx][kk] = static_cast<int8_t>(sl);
-      }
-    }
-    __syncthreads();
-    for (int cc = ty; cc < 32; cc += 8) {
-      const int64_t nn = static_cast<int64_t>(blockIdx.x) * 32 + cc;
-      if (nn < N)
-        for (int p = 0; p < NS; ++p) S[(static_cast<int64_t>(p) * N + nn) * KP + k0 + tx] = tile[p][cc][tx];
-    }
-    __syncthreads();
+  // rows (p, column) of KW bytes, stored as 32-bit words (consecutive threads, consecutive words)
+  for (int idx = threadIdx.x; idx < NS * 32 * WPR; idx += 256) {
+    const int row = idx / WPR, w = idx % WPR;
+    const int p = row / 32, c = row % 32;
+    const int64_t nn = static_cast<int64_t>(blockIdx.x) * 32 + c;
+    if (nn < N)
+      *reinterpret_cast<uint32_t*>(S + (static_cast<int64_t>(p) * N + nn) * KP + k0 + 4 * w) =
+          *reinterpret_cast<const uint32_t*>(&tile[p][c][4 * w]);
   }
 }
 
@@ -504,8 +541,25 @@ int split_rows_any(cudaStream_t s, const double* X, int64_t ldx, int64_t R, int6
 template <int NS>
 int split_cols_any(cudaStream_t s, const double* Y, int64_t ldy, int64_t K, int64_t N, int64_t KP, int8_t* S, int* e) {
   if (N <= 0) return GPTQ_OK;
-  split_cols_kernel<NS><<<static_cast<unsigned>((N + 31) / 32), 256, 0, s>>>(Y, ldy, K, N, KP, S, e);
-  return after_launch();
+  if (KP % 64 != 0) return GPTQ_ERR_UNSUPPORTED;
+  const unsigned gx = static_cast<unsigned>((N + 31) / 32);
+  col_exp_init_kernel<<<static_cast<unsigned>((N + 255) / 256), 256, 0, s>>>(e, N);
+  GPTQ_TRY(after_launch());
+  if (K > 0) {
+    col_exp_kernel<<<dim3(gx, static_cast<unsigned>((K + CE_ROWS - 1) / CE_ROWS)), 256, 0, s>>>(Y, ldy, K, N, e);
+    GPTQ_TRY(after_launch());
+  }
+  // KP is a multiple of 64: 128-wide chunks, and one 64-wide chunk for an odd remainder
+  const int64_t full = KP / CS_K;
+  if (full > 0) {
+    col_slices_kernel<NS, CS_K><<<dim3(gx, static_cast<unsigned>(full)), 256, 0, s>>>(Y, ldy, K, N, KP, 0, S, e);
+    GPTQ_TRY(after_launch());
+  }
+  if (KP % CS_K != 0) {
+    col_slices_kernel<NS, 64><<<dim3(gx, 1), 256, 0, s>>>(Y, ldy, K, N, KP, full * CS_K, S, e);
+    GPTQ_TRY(after_launch());
+  }
+  return GPTQ_OK;
 }
 
 template <int NS, int BN, int NBUF, int CR>

@@ -329,8 +329,9 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
 //  * float16: 0x6400 | q is the half 1024 + q (exact for q < 1024); subtracting 1024 + z
 //    leaves q - z exactly, and one half multiply by s rounds the exact product once, to
 //    nearest even: round16(s * (q - z)), two codes per instruction.
-//  * bfloat16: the same in fp32 (0x4B000000 | q is 2^23 + q): q - z and s * (q - z) are
-//    exact in fp32 (a 19-bit product), then one rounding to bfloat16.
+//  * bfloat16: the same with bf16 pairs, the scale split in two bf16 parts so that one
+//    fused multiply-add rounds the exact product once (8-bit codes: in fp32, 0x4B000000 | q
+//    being 2^23 + q, then one rounding to bfloat16).
 template <typename T>
 struct PairDeq;
 template <>
@@ -350,18 +351,32 @@ struct PairDeq<__half> {
 };
 template <>
 struct PairDeq<__nv_bfloat16> {
-  float2 s2, zb2;
+  // codes of up to 4 bits: s = s_hi + s_lo with s_hi = bf16(s) and s_lo (at most 3 bits) both
+  // exact in bf16; 0x4300 | q is the bf16 128 + q, so d = q - z is exact, s_lo d is exact (at
+  // most 7 bits) and one bf16 FMA s_hi d + s_lo d rounds the exact product once
+  __nv_bfloat162 shi2, slo2, zb2;
+  // 8-bit codes (q - z needs 9 bits): the fp32 route, exact up to one rounding to bf16
+  float2 s2, zf2;
   __device__ __forceinline__ void set(float s, int z) {
+    const __nv_bfloat16 hi = __float2bfloat16_rn(s);
+    shi2 = __bfloat162bfloat162(hi);
+    slo2 = __bfloat162bfloat162(__float2bfloat16_rn(s - __bfloat162float(hi)));
+    zb2 = __bfloat162bfloat162(__float2bfloat16_rn(128.f + static_cast<float>(z)));
     s2 = make_float2(s, s);
-    zb2 = make_float2(8388608.f + static_cast<float>(z), 8388608.f + static_cast<float>(z));
+    zf2 = make_float2(8388608.f + static_cast<float>(z), 8388608.f + static_cast<float>(z));
   }
   template <int BITS>
   __device__ __forceinline__ float2 pair(uint32_t w, int i) const {
     constexpr uint32_t m = (1u << BITS) - 1u;
-    const uint32_t lo = (w >> (i * BITS)) & m, hi = (w >> (i * BITS + 16)) & m;
-    const float2 q = make_float2(__uint_as_float(0x4B000000u | lo), __uint_as_float(0x4B000000u | hi));
-    const __nv_bfloat162 b = __float22bfloat162_rn(mul2(sub2(q, zb2), s2));
-    return __bfloat1622float2(b);
+    if constexpr (BITS <= 4) {
+      const uint32_t h = ((w >> (i * BITS)) & ((m << 16) | m)) | 0x43004300u;
+      const __nv_bfloat162 d = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&h), zb2);
+      return __bfloat1622float2(__hfma2(shi2, d, __hmul2(slo2, d)));
+    } else {
+      const uint32_t lo = (w >> (i * BITS)) & m, hi = (w >> (i * BITS + 16)) & m;
+      const float2 q = make_float2(__uint_as_float(0x4B000000u | lo), __uint_as_float(0x4B000000u | hi));
+      return __bfloat1622float2(__float22bfloat162_rn(mul2(sub2(q, zf2), s2)));
+    }
   }
 };
 
