@@ -4,10 +4,12 @@
 //
 // Lanes are created once per device and priority class and kept on a free list, so a call
 // pays no stream creation; concurrent calls from several host threads lease disjoint
-// lanes.  A lease forks every lane from the caller's stream (the lane starts after all
+// lanes, and a lease takes only lanes whose earlier work has drained (the pool grows to the
+// largest number of lanes in flight at once).  A lease forks every lane from the caller's stream (the lane starts after all
 // work already queued there) and, when it ends, makes the caller's stream wait for all
 // work issued on its lanes, on error paths too, so stream-ordered frees of the call's
 // workspace on the caller's stream never overtake a lane.
+#include <cstddef>
 #include <map>
 #include <mutex>
 #include <vector>
@@ -56,11 +58,20 @@ int LaneLease::acquire(int count, const LanePrio* prio) {
   for (int i = 0; i < count; ++i) {
     Lane* l = nullptr;
     {
+      // Only a lane whose previous lease has drained: a lane handed back by a call that the
+      // host has finished issuing may still hold queued work, and this lease's work would
+      // wait behind it (correct, but two concurrent users of the library would run one
+      // after the other).  Without an idle lane, a new one is created.
       std::lock_guard<std::mutex> lk(g_lane_mu);
       auto& v = g_lane_free[{dev_, static_cast<int>(prio[i])}];
-      if (!v.empty()) {
-        l = v.back();
-        v.pop_back();
+      for (size_t k = v.size(); k-- > 0;) {
+        const cudaError_t q = cudaEventQuery(v[k]->join);
+        if (q == cudaSuccess) {
+          l = v[k];
+          v.erase(v.begin() + static_cast<std::ptrdiff_t>(k));
+          break;
+        }
+        if (q == cudaErrorNotReady) cudaGetLastError();  // "not yet" is not an error: clear it
       }
     }
     if (!l) GPTQ_TRY(create_lane(prio[i], &l));
