@@ -258,9 +258,8 @@ def run_native(args, world, rank, local):
     cols = layer_columns(cfg)
     value = cols * world / (ms / 1e3)
     work = algorithmic_work(cfg, T)
-    h_ms = statistics.mean(p.hessian_ms for p in phase)
     fs_ms = statistics.mean(p.factor_sweep_ms for p in phase)
-    spread = {"hessian_ms": [round(f(p.hessian_ms for p in phase), 3) for f in (min, statistics.median, max)],
+    spread = {"step_ms": [round(f(p.total_ms for p in phase), 3) for f in (min, statistics.median, max)],
               "factor_and_sweep_ms": [round(f(p.factor_sweep_ms for p in phase), 3)
                                       for f in (min, statistics.median, max)]}
     # factor and sweep apart: the timed steps themselves in the two-phase route, else a few
@@ -270,9 +269,12 @@ def run_native(args, world, rank, local):
         attrib = [step(timing=True, pipelined=False)[1] for _ in range(max(args.phase_steps, 1))]
     f_ms = statistics.mean(p.factor_ms for p in attrib)
     s_ms = statistics.mean(p.sweep_ms for p in attrib)
+    # the Hessian phase and its launches from the two-phase steps, where nothing overlaps them
+    h_ms = statistics.mean(p.hessian_ms for p in attrib)
+    spread["two_phase_hessian_ms"] = [round(f(p.hessian_ms for p in attrib), 3) for f in (min, statistics.median, max)]
     spread["two_phase_factor_ms"] = [round(f(p.factor_ms for p in attrib), 3) for f in (min, statistics.median, max)]
     spread["two_phase_sweep_ms"] = [round(f(p.sweep_ms for p in attrib), 3) for f in (min, statistics.median, max)]
-    launch_ms = [statistics.mean(p.hessian_launch_ms[i] for p in phase) for i in range(len(cfg.hessian_n))]
+    launch_ms = [statistics.mean(p.hessian_launch_ms[i] for p in attrib) for i in range(len(cfg.hessian_n))]
     h_flops = sum(work["hessian_flops"])
     h_tflops = h_flops / (sum(launch_ms) / 1e3) / 1e12
     per_launch = [work["hessian_flops"][i] / (launch_ms[i] / 1e3) / 1e12 for i in range(len(launch_ms))]
@@ -309,7 +311,10 @@ def run_native(args, world, rank, local):
                                       "boost clock, not measured on this part"},
         "factor_and_sweep": {"ms": round(fs_ms, 3), "pipelined": not args.two_phase,
                              "two_phase_ms": round(f_ms + s_ms, 3),
-                             "note": "timed steps; factor and sweep below come from two-phase steps"
+                             "note": ("timed steps, two phases" if args.two_phase else
+                                      "timed steps: from the largest Hessian's completion to the end, overlapping "
+                                      "the other Hessians' accumulation") +
+                                     "; the hessian, factor and sweep entries come from two-phase steps"
                                      + ("" if args.two_phase else " run after the timed region")},
         "factor": {"ms": round(f_ms, 3), "tflops_fp64": round(f_tflops, 2),
                    "frac_of_fp64_peak": round(f_tflops / fp64_peak, 4)},
@@ -698,7 +703,7 @@ def run_cpu_full_layer(args):
 
 def run_qlinear(args):
     """The linear on the quantized checkpoint (4-bit, group 128; act order, and for decoding also
-    without it), measured alone on Llama-shaped weights quantized by the library itself: the decode kernel (M = 1 and 4 rows; HBM-bound: bytes =
+    without it and with the act-order checkpoint's inputs sorted by group), measured alone on Llama-shaped weights quantized by the library itself: the decode kernel (M = 1 and 4 rows; HBM-bound: bytes =
     packed codes + fp16 scales + packed zero points + g_idx + X + Y) against the measured
     copy bandwidth, the dequantization (bytes = the checkpoint read + the 16-bit weight
     written) likewise, and the tensor-core GEMM (2 M N K flops) against the measured bf16
@@ -784,7 +789,8 @@ def run_qlinear(args):
         G = ck["scales"].shape[0]
         wbytes = n_in * n_out * bits // 8 + G * n_out * (2 + bits / 8) + n_in * 4
         row = {"shape": name, "n_in": n_in, "n_out": n_out, "weight_bytes": int(wbytes)}
-        for tag, c in (("", ck), ("_monotone_groups", ck_mono)):
+        ck_re = gq.reorder_act_order(ck, bits)  # the act-order checkpoint with its inputs sorted by group
+        for tag, c in (("", ck), ("_monotone_groups", ck_mono), ("_act_order_reordered", ck_re)):
             for M in (1, 4):
                 X = torch.randn(M, n_in, device=dev).to(torch.bfloat16)
                 Y = torch.empty(M, n_out, device=dev, dtype=torch.bfloat16)

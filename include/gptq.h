@@ -208,8 +208,15 @@ int gptq_quantize_layer_factored(const void* W, int w_dtype, int64_t n_out, int6
  * still in progress.  All streams fork from `stream` and join back into it.  Workspace
  * (stream-ordered, from the library's pool): the factor workspaces of all Hessians plus
  * 17 * n_out[j] * n_in bytes per linear, held until the call returns.
+ * hessian_ready: optional host array of n_hessians CUDA event handles (cudaEvent_t), NULL
+ *       entries allowed: Hessian i's factor also waits for hessian_ready[i].  Every chain
+ *       already starts after the work queued on `stream` at the call; the events let a
+ *       caller accumulate some Hessians on other streams (for instance the largest on
+ *       `stream` and the rest on a side stream), so that a factor starts as soon as its own
+ *       Hessian is complete.  Workspace is allocated on `stream`, so a Hessian accumulated on
+ *       another stream must not depend on this call.
  * statuses: optional host array of n_linears ints: the Hessian's factor status (NOT_PD)
- * when that failed, else the linear's sweep status.  Returns GPTQ_OK when every linear
+ *       when that failed, else the linear's sweep status.  Returns GPTQ_OK when every linear
  * succeeded, else the first failing linear's status.  n_hessians or n_linears <= 0, a NULL
  * array or pointer, hessian_of out of range -> INVALID_ARG; argument rules of
  * gptq_factor_hessians and gptq_quantize_layer otherwise.  Blocking.
@@ -220,7 +227,7 @@ int gptq_quantize_linears(int n_hessians, const float* const* H, const int64_t* 
                           const int* hessian_of, int bits, int group_size, int sym,
                           int static_groups, int blocksize, int32_t* const* qweight,
                           float* const* scales, int32_t* const* zeros, int32_t* const* g_idx,
-                          void* stream, int* statuses);
+                          void* const* hessian_ready, void* stream, int* statuses);
 
 /*
  * Checkpoint form of one quantized linear: half-precision scales and packed zero points.
@@ -269,6 +276,9 @@ int gptq_dequantize_weight(const int32_t* qweight, const int32_t* qzeros, const 
  * X [M, n_in] fp16 or bf16 (x_dtype), Y [M, n_out] of the same dtype; M >= 0 (0: no-op,
  * X and Y may then be NULL).
  * Weight arguments as in gptq_dequantize_weight.
+ * x_perm: NULL, or [n_in] int32 (16-byte aligned): the checkpoint's row k of codes belongs to
+ *       input x_perm[k], i.e. Y = X[:, x_perm] * round16(W_hat)^T (the form that
+ *       gptq_reorder_act_order produces; an entry outside [0, n_in) is clamped into it).
  * M <= 4 (decoding): one pass over the packed weights, dequantized in registers, K split
  * over CTAs and the splits added in a fixed order (deterministic).  M > 4: the weights are
  * dequantized once into a 16-bit workspace (library pool, n_in*n_out*2 bytes) and
@@ -278,7 +288,30 @@ int gptq_dequantize_weight(const int32_t* qweight, const int32_t* qzeros, const 
  */
 int gptq_quantized_linear(const void* X, int x_dtype, int64_t M, int64_t n_in, const int32_t* qweight,
                           const int32_t* qzeros, const uint16_t* scales_f16, const int32_t* g_idx,
-                          int64_t groups, int64_t n_out, int bits, void* Y, void* stream);
+                          const int32_t* x_perm, int64_t groups, int64_t n_out, int bits, void* Y,
+                          void* stream);
+
+/*
+ * Reorder an act-order checkpoint so that its g_idx runs in order.  With desc_act the
+ * checkpoint keeps the codes in the original input order and g_idx names each input's group
+ * (AutoGPTQ examples guide §1.4, desc_act; the group of an input is its position in the
+ * quantization order divided by group_size), so the inputs of one 32-bit word belong to
+ * different groups.  This call sorts the inputs by (g_idx, index), stably:
+ *   x_perm[k'] = the input with the k'-th smallest (g_idx[k], k),
+ *   g_idx_out[k'] = g_idx[x_perm[k']] (non-decreasing),
+ *   qweight_out holds at row k' the code of input x_perm[k'] (same packing).
+ * qzeros and scales are unchanged.  gptq_quantized_linear on (qweight_out, g_idx_out,
+ * x_perm) then gives the same product as on the original checkpoint (Y = X W_hat^T), its
+ * fp32 sums taken in another order; gptq_dequantize_weight on it gives W_hat[:, x_perm].
+ * qweight [n_in*bits/32, n_out] and g_idx [n_in] read-only; qweight_out (same shape),
+ * g_idx_out and x_perm ([n_in] int32) written, none aliasing an input.  g_idx entries outside
+ * [0, groups) are clamped.  bits 2, 4, 8 (3 -> UNSUPPORTED); n_in % 64 == 0 and n_in <= 65536,
+ * else UNSUPPORTED.  Asynchronous on `stream`; the sort runs in one CTA (a preparation
+ * step, once per checkpoint).
+ */
+int gptq_reorder_act_order(const int32_t* qweight, const int32_t* g_idx, int64_t groups, int64_t n_in,
+                           int64_t n_out, int bits, int32_t* qweight_out, int32_t* g_idx_out,
+                           int32_t* x_perm, void* stream);
 
 /*
  * Forward pieces of a Llama-style decoder layer, used to quantize its linears in execution

@@ -21,6 +21,7 @@ from .api import (  # noqa: F401
     quantize_layer_factored,
     quantize_linears,
     quantized_linear,
+    reorder_act_order,
 )
 
 __version__ = "0.1.0"

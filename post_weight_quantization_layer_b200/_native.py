@@ -53,12 +53,14 @@ _SIGNATURES = {
                                       ctypes.POINTER(c_void_p), c_int, ctypes.POINTER(c_i64), ctypes.POINTER(c_int),
                                       c_int, c_int, c_int, c_int, c_int, ctypes.POINTER(c_void_p),
                                       ctypes.POINTER(c_void_p), ctypes.POINTER(c_void_p), ctypes.POINTER(c_void_p),
-                                      c_void_p, ctypes.POINTER(c_int)]),
+                                      ctypes.POINTER(c_void_p), c_void_p, ctypes.POINTER(c_int)]),
     "gptq_export_layer": (c_int, [c_void_p, c_void_p, c_i64, c_i64, c_int, c_void_p, c_void_p, c_void_p]),
     "gptq_dequantize_weight": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_i64, c_i64, c_i64, c_int, c_int,
                                        c_void_p, c_void_p]),
-    "gptq_quantized_linear": (c_int, [c_void_p, c_int, c_i64, c_i64, c_void_p, c_void_p, c_void_p, c_void_p, c_i64,
-                                      c_i64, c_int, c_void_p, c_void_p]),
+    "gptq_quantized_linear": (c_int, [c_void_p, c_int, c_i64, c_i64, c_void_p, c_void_p, c_void_p, c_void_p,
+                                      c_void_p, c_i64, c_i64, c_int, c_void_p, c_void_p]),
+    "gptq_reorder_act_order": (c_int, [c_void_p, c_void_p, c_i64, c_i64, c_i64, c_int, c_void_p, c_void_p, c_void_p,
+                                       c_void_p]),
     "gptq_test_wait_expiry": (c_int, [c_int, ctypes.c_uint32]),
     "gptq_rmsnorm": (c_int, [c_void_p, c_int, c_i64, c_i64, c_void_p, c_float, c_void_p, c_void_p]),
     "gptq_rope": (c_int, [c_void_p, c_int, c_i64, c_int, c_int, c_int, ctypes.c_double, c_void_p]),

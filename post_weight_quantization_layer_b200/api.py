@@ -207,12 +207,14 @@ def quantize_layer_factored(W, U, perm, bits=4, group_size=128, sym=True, static
 
 
 def quantize_linears(Hs, linears, bits=4, group_size=128, damp_percent=0.01, sym=True, desc_act=False,
-                      static_groups=False, blocksize=128, stream=None):
+                      static_groups=False, blocksize=128, stream=None, ready=None):
     """Factor every Hessian in Hs and quantize every linear in one pipelined call.
 
     Hs:      list of [n, n] float32 Hessians.
     linears: list of (W, h) pairs: W [n_out, n_in] weight (all of one dtype) whose input has
              Hessian Hs[h].
+    ready:   optional list (one per Hessian) of recorded torch.cuda.Event or None: Hessian i's
+             factor also waits for ready[i] (for Hessians accumulated on another stream).
     Returns ([(U, perm) per Hessian], [QuantResult per linear]): bit-identical to
     factor_hessians followed by quantize_layer_factored per linear.  Raises GPTQError naming
     the first linear that failed."""
@@ -235,6 +237,8 @@ def quantize_linears(Hs, linears, bits=4, group_size=128, damp_percent=0.01, sym
             raise ValueError(f"linear {j}: n_in {n_in} does not match its Hessian's order {Hs[h].shape[0]}")
         outs.append(_outputs(n_out, n_in, bits, group_size, W.device, None))
         hidx.append(h)
+    if ready is not None and len(ready) != len(Hs):
+        raise ValueError("ready needs one entry (an event or None) per Hessian")
     _need_cuda(*Hs, *[W for W, _ in linears])
     factors = [(torch.empty(H.shape[0], H.shape[0], dtype=torch.float64, device=H.device),
                 torch.empty(H.shape[0], dtype=torch.int32, device=H.device)) for H in Hs]
@@ -248,7 +252,8 @@ def quantize_linears(Hs, linears, bits=4, group_size=128, damp_percent=0.01, sym
         (ctypes.c_int64 * kl)(*[W.shape[0] for W, _ in linears]), (ctypes.c_int * kl)(*hidx), bits, group_size,
         int(bool(sym)), int(bool(static_groups)), blocksize, al(*[o[0].data_ptr() for o in outs]),
         al(*[o[1].data_ptr() for o in outs]), al(*[o[2].data_ptr() for o in outs]),
-        al(*[o[3].data_ptr() for o in outs]), _stream(stream), st_arr)
+        al(*[o[3].data_ptr() for o in outs]),
+        None if ready is None else ah(*[None if e is None else e.cuda_event for e in ready]), _stream(stream), st_arr)
     if st != OK:
         bad = next((j for j in range(kl) if st_arr[j] != OK), None)
         _check(st, "gptq_quantize_linears" + (f" (linear {bad})" if bad is not None else ""))
@@ -272,6 +277,9 @@ def _checkpoint(ck, bits):
     _need(qz, "qzeros", (torch.int32,), (G, n_out * bits // 32))
     _need(sc, "scales", (torch.float16,), (G, n_out))
     _need(gi, "g_idx", (torch.int32,), (n_in,))
+    xp = ck.get("x_perm") if isinstance(ck, dict) else None
+    if xp is not None:
+        _need(xp, "x_perm", (torch.int32,), (n_in,))
     return qw, qz, sc, gi, G, n_in, n_out
 
 
@@ -299,10 +307,29 @@ def quantized_linear(X, ck, bits=4, out=None, stream=None):
     if out is None:
         out = torch.empty(M, n_out, dtype=X.dtype, device=X.device)
     _need(out, "out", (X.dtype,), (M, n_out))
-    _need_cuda(X, out, qw, qz, sc, gi)
-    st = lib().gptq_quantized_linear(_ptr(X), _DTYPE[X.dtype], M, n_in, _ptr(qw), _ptr(qz), _ptr(sc), _ptr(gi), G,
-                                     n_out, bits, _ptr(out), _stream(stream))
+    xp = ck.get("x_perm")
+    _need_cuda(X, out, qw, qz, sc, gi, *([xp] if xp is not None else []))
+    st = lib().gptq_quantized_linear(_ptr(X), _DTYPE[X.dtype], M, n_in, _ptr(qw), _ptr(qz), _ptr(sc), _ptr(gi),
+                                     None if xp is None else _ptr(xp), G, n_out, bits, _ptr(out), _stream(stream))
     _check(st, "gptq_quantized_linear")
+    return out
+
+
+def reorder_act_order(ck, bits=4, stream=None):
+    """An act-order checkpoint with its inputs sorted by group (gptq_reorder_act_order): a new
+    dict with qweight and g_idx reordered, qzeros and scales shared, and x_perm (row k of the
+    codes belongs to input x_perm[k]).  quantized_linear gives the same product on it, with
+    every word of codes in one group."""
+    qw, qz, sc, gi, G, n_in, n_out = _checkpoint(ck, bits)
+    if ck.get("x_perm") is not None:
+        raise ValueError("checkpoint is already reordered")
+    _need_cuda(qw, gi)
+    qw2, gi2, xp = torch.empty_like(qw), torch.empty_like(gi), torch.empty_like(gi)
+    st = lib().gptq_reorder_act_order(_ptr(qw), _ptr(gi), G, n_in, n_out, bits, _ptr(qw2), _ptr(gi2), _ptr(xp),
+                                      _stream(stream))
+    _check(st, "gptq_reorder_act_order")
+    out = dict(ck)
+    out.update(qweight=qw2, g_idx=gi2, x_perm=xp)
     return out
 
 

@@ -366,8 +366,8 @@ int gptq_quantize_linears(int n_hessians, const float* const* H, const int64_t* 
                           int desc_act, double* const* U, int32_t* const* perm, int n_linears,
                           const void* const* W, int w_dtype, const int64_t* n_out, const int* hessian_of, int bits,
                           int group_size, int sym, int static_groups, int blocksize, int32_t* const* qweight,
-                          float* const* scales, int32_t* const* zeros, int32_t* const* g_idx, void* stream,
-                          int* statuses) {
+                          float* const* scales, int32_t* const* zeros, int32_t* const* g_idx,
+                          void* const* hessian_ready, void* stream, int* statuses) {
   if (n_hessians <= 0 || n_linears <= 0 || !H || !n_in || !U || !perm || !W || !n_out || !hessian_of || !qweight ||
       !scales || !zeros || !g_idx)
     return GPTQ_ERR_INVALID_ARG;
@@ -408,6 +408,11 @@ int gptq_quantize_linears(int n_hessians, const float* const* H, const int64_t* 
     // that reads it.  The sub-leases end before the chain lease (reverse declaration order).
     LaneLease chains(s);
     GPTQ_TRY(chains.acquire(n_hessians, prio.data()));
+    // A Hessian finished on another stream: its chain also waits for the caller's event.
+    if (hessian_ready)
+      for (int i = 0; i < n_hessians; ++i)
+        if (hessian_ready[i])
+          GPTQ_CUDA(cudaStreamWaitEvent(chains[i].st, static_cast<cudaEvent_t>(hessian_ready[i]), 0));
     std::vector<std::unique_ptr<LaneLease>> subs;
     for (int i = 0; i < n_hessians; ++i) {
       const int64_t n = n_in[i];

@@ -392,7 +392,8 @@ __global__ void __launch_bounds__(GV_THREADS, 2) gemv_kernel(const T* __restrict
                                                           const int32_t* __restrict__ qweight,
                                                           const int32_t* __restrict__ qzeros,
                                                           const __half* __restrict__ scales,
-                                                          const int32_t* __restrict__ g_idx, int G, int64_t N,
+                                                          const int32_t* __restrict__ g_idx,
+                                                          const int32_t* __restrict__ x_perm, int G, int64_t N,
                                                           int kchunk, float* __restrict__ partial) {
   constexpr int FPW = 32 / BITS;
   constexpr int HP = FPW / 2;  // code pairs per word
@@ -412,7 +413,10 @@ __global__ void __launch_bounds__(GV_THREADS, 2) gemv_kernel(const T* __restrict
     const int r = e / FPW, f = e % FPW;
     float* slot = reinterpret_cast<float*>(xs + r * HP + (f % HP)) + (f / HP);
 #pragma unroll
-    for (int m = 0; m < MM; ++m) slot[m * kchunk] = to_f32<T>(X[m * K + klo + e]);
+    // the input behind row k of the codes (clamped: a malformed permutation reads inside X)
+    const int64_t kx = x_perm ? min(max(static_cast<int64_t>(__ldg(x_perm + klo + e)), int64_t(0)), K - 1) : klo + e;
+#pragma unroll
+    for (int m = 0; m < MM; ++m) slot[m * kchunk] = to_f32<T>(X[m * K + kx]);
   }
   __syncthreads();
   for (int r = tid; r < rows; r += GV_THREADS) {
@@ -432,7 +436,7 @@ __global__ void __launch_bounds__(GV_THREADS, 2) gemv_kernel(const T* __restrict
   if (n < N) {
     const int64_t zw = N * BITS / 32;
     const int zshift = static_cast<int>((n * BITS) % 32);
-    int gcur = -1;
+    int gcur = -1, gpair = -1;  // group of sc/zc, group of pd
     PairDeq<T> pd[4];
     float sc[4];
     int zc[4];
@@ -447,17 +451,19 @@ __global__ void __launch_bounds__(GV_THREADS, 2) gemv_kernel(const T* __restrict
       sc[3] = __high2float(s23);
       const uint32_t zword = static_cast<uint32_t>(__ldg(qzeros + static_cast<int64_t>(g) * zw + (n * BITS) / 32));
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        zc[j] = static_cast<int>((zword >> (zshift + j * BITS)) & MASK);
-        pd[j].set(sc[j], zc[j]);
-      }
+      for (int j = 0; j < 4; ++j) zc[j] = static_cast<int>((zword >> (zshift + j * BITS)) & MASK);
     };
     auto row_math = [&](int r, const int4 w4) {
       const uint32_t wv[4] = {static_cast<uint32_t>(w4.x), static_cast<uint32_t>(w4.y), static_cast<uint32_t>(w4.z),
                               static_cast<uint32_t>(w4.w)};
       const int g = rg[r];
       if (g >= 0) {
-        if (g != gcur) load_group(g);
+        if (g != gpair) {
+          if (g != gcur) load_group(g);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) pd[j].set(sc[j], zc[j]);
+          gpair = g;
+        }
 #pragma unroll
         for (int i = 0; i < HP; ++i) {
           float2 xp[MM];
@@ -520,6 +526,106 @@ __global__ void __launch_bounds__(GV_THREADS, 2) gemv_kernel(const T* __restrict
       partial[(static_cast<int64_t>(blockIdx.y) * M + m) * N + nn] = t;
     }
   }
+}
+
+// ------------------------------------------------------------------ act-order reordering
+// A checkpoint quantized with act order stores its codes in the original input order, with
+// g_idx naming each input's group; the inputs of a 32-bit word then belong to different
+// groups.  Reordering the inputs by group (and gathering X by the same permutation) gives a
+// checkpoint whose g_idx runs in order, which the decode kernel dequantizes two codes at a
+// time; the product is the same sum over the inputs in another order.
+//
+// perm[k'] = the input with the k'-th smallest (g_idx, index): one CTA of 1024 threads, the
+// group sizes in shared memory, their exclusive scan, then the inputs in chunks of 1024 in
+// increasing index, each placed at its group's running offset plus its rank among the chunk's
+// inputs of the same group (stable, deterministic).
+constexpr int RO_THREADS = 1024;
+__global__ void __launch_bounds__(RO_THREADS) sort_by_group_kernel(const int32_t* __restrict__ g_idx, int K, int G,
+                                                                   int32_t* __restrict__ perm,
+                                                                   int32_t* __restrict__ g_sorted) {
+  extern __shared__ int ro_sm[];
+  int* off = ro_sm;             // [G] group sizes, then running offsets
+  int* gch = ro_sm + G;         // [RO_THREADS] groups of the current chunk
+  int* part = gch + RO_THREADS; // [RO_THREADS] per-thread partial sums of the scan
+  const int tid = threadIdx.x;
+  for (int g = tid; g < G; g += RO_THREADS) off[g] = 0;
+  __syncthreads();
+  for (int k = tid; k < K; k += RO_THREADS) atomicAdd(&off[clamp_group(g_idx[k], G)], 1);
+  __syncthreads();
+  // exclusive scan: each thread a contiguous range, then the range totals by thread 0
+  const int per = (G + RO_THREADS - 1) / RO_THREADS;
+  const int lo = min(G, tid * per), hi = min(G, lo + per);
+  int sum = 0;
+  for (int g = lo; g < hi; ++g) sum += off[g];
+  part[tid] = sum;
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int t = 0; t < RO_THREADS; ++t) {
+      const int v = part[t];
+      part[t] = run;
+      run += v;
+    }
+  }
+  __syncthreads();
+  int run = part[tid];
+  for (int g = lo; g < hi; ++g) {
+    const int v = off[g];
+    off[g] = run;
+    run += v;
+  }
+  __syncthreads();
+  for (int c0 = 0; c0 < K; c0 += RO_THREADS) {
+    const int k = c0 + tid;
+    const int g = k < K ? clamp_group(g_idx[k], G) : -1;
+    gch[tid] = g;
+    __syncthreads();
+    int rank = 0;
+    bool last = true;
+    if (g >= 0) {
+      for (int j = 0; j < RO_THREADS; ++j) {
+        const int gj = gch[j];
+        rank += (j < tid && gj == g) ? 1 : 0;
+        last = last && !(j > tid && gj == g);
+      }
+      const int pos = off[g] + rank;
+      perm[pos] = k;
+      g_sorted[pos] = g;
+    }
+    __syncthreads();  // every rank and offset read before the offsets move on
+    if (g >= 0 && last) off[g] += rank + 1;  // the group's last input of the chunk
+    __syncthreads();
+  }
+}
+
+// Word row r' of the reordered codes holds inputs perm[r' FPW .. r' FPW + FPW - 1].
+template <int BITS>
+__global__ void reorder_codes_kernel(const int32_t* __restrict__ qweight, const int32_t* __restrict__ perm,
+                                     int64_t rows, int64_t N, int32_t* __restrict__ out) {
+  constexpr int FPW = 32 / BITS;
+  constexpr uint32_t MASK = (1u << BITS) - 1u;
+  const int64_t n = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t r = blockIdx.y;
+  if (n >= N || r >= rows) return;
+  uint32_t w = 0;
+#pragma unroll
+  for (int f = 0; f < FPW; ++f) {
+    const int k = perm[r * FPW + f];
+    const uint32_t src = static_cast<uint32_t>(__ldg(qweight + static_cast<int64_t>(k / FPW) * N + n));
+    w |= ((src >> ((k % FPW) * BITS)) & MASK) << (f * BITS);
+  }
+  out[r * N + n] = static_cast<int32_t>(w);
+}
+
+// X'[m, k'] = X[m, perm[k']] for the tensor-core path.
+template <typename T>
+__global__ void gather_cols_kernel(const T* __restrict__ X, const int32_t* __restrict__ perm, int64_t M, int64_t K,
+                                   T* __restrict__ Xp) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= M * K) return;
+  const int64_t m = i / K, k = i % K;
+  const int64_t kx = min(max(static_cast<int64_t>(perm[k]), int64_t(0)), K - 1);
+  Xp[i] = X[m * K + kx];
 }
 
 // Y[m, n] = sum over K splits of partial[s, m, n], in split order.
@@ -597,7 +703,7 @@ int dequant_any(int bits, const int32_t* qw, const int32_t* qz, const __half* sc
 
 template <int BITS, typename T, int MM>
 int launch_gemv(const T* X, int M, int64_t K, const int32_t* qw, const int32_t* qz, const __half* sc,
-                const int32_t* gi, int G, int64_t N, T* Y, cudaStream_t s) {
+                const int32_t* gi, const int32_t* xp, int G, int64_t N, T* Y, cudaStream_t s) {
   // K split so that about four CTAs per SM stream the weights; every split a multiple of
   // 64 columns (whole words for every bit width).
   const int64_t nblk = (N + GV_N - 1) / GV_N;
@@ -611,7 +717,7 @@ int launch_gemv(const T* X, int M, int64_t K, const int32_t* qw, const int32_t* 
   float* partial = nullptr;
   GPTQ_TRY(pool_alloc(reinterpret_cast<void**>(&partial), static_cast<size_t>(S) * M * N * 4, s));
   gemv_kernel<BITS, T, MM><<<dim3(static_cast<unsigned>(nblk), static_cast<unsigned>(S)), GV_THREADS, smem, s>>>(
-      X, M, K, qw, qz, sc, gi, G, N, static_cast<int>(kchunk), partial);
+      X, M, K, qw, qz, sc, gi, xp, G, N, static_cast<int>(kchunk), partial);
   int st = after_launch();
   if (st == GPTQ_OK) {
     const int64_t cnt = static_cast<int64_t>(M) * N;
@@ -624,21 +730,21 @@ int launch_gemv(const T* X, int M, int64_t K, const int32_t* qw, const int32_t* 
 
 template <int BITS, typename T>
 int gemv_rows(const T* X, int M, int64_t K, const int32_t* qw, const int32_t* qz, const __half* sc,
-              const int32_t* gi, int G, int64_t N, T* Y, cudaStream_t s) {
+              const int32_t* gi, const int32_t* xp, int G, int64_t N, T* Y, cudaStream_t s) {
   switch (M) {
-    case 1: return launch_gemv<BITS, T, 1>(X, M, K, qw, qz, sc, gi, G, N, Y, s);
-    case 2: return launch_gemv<BITS, T, 2>(X, M, K, qw, qz, sc, gi, G, N, Y, s);
-    case 3: return launch_gemv<BITS, T, 3>(X, M, K, qw, qz, sc, gi, G, N, Y, s);
-    default: return launch_gemv<BITS, T, 4>(X, M, K, qw, qz, sc, gi, G, N, Y, s);
+    case 1: return launch_gemv<BITS, T, 1>(X, M, K, qw, qz, sc, gi, xp, G, N, Y, s);
+    case 2: return launch_gemv<BITS, T, 2>(X, M, K, qw, qz, sc, gi, xp, G, N, Y, s);
+    case 3: return launch_gemv<BITS, T, 3>(X, M, K, qw, qz, sc, gi, xp, G, N, Y, s);
+    default: return launch_gemv<BITS, T, 4>(X, M, K, qw, qz, sc, gi, xp, G, N, Y, s);
   }
 }
 
 template <typename T>
 int gemv_any(int bits, const T* X, int M, int64_t K, const int32_t* qw, const int32_t* qz, const __half* sc,
-             const int32_t* gi, int G, int64_t N, T* Y, cudaStream_t s) {
-  if (bits == 2) return gemv_rows<2, T>(X, M, K, qw, qz, sc, gi, G, N, Y, s);
-  if (bits == 4) return gemv_rows<4, T>(X, M, K, qw, qz, sc, gi, G, N, Y, s);
-  return gemv_rows<8, T>(X, M, K, qw, qz, sc, gi, G, N, Y, s);
+             const int32_t* gi, const int32_t* xp, int G, int64_t N, T* Y, cudaStream_t s) {
+  if (bits == 2) return gemv_rows<2, T>(X, M, K, qw, qz, sc, gi, xp, G, N, Y, s);
+  if (bits == 4) return gemv_rows<4, T>(X, M, K, qw, qz, sc, gi, xp, G, N, Y, s);
+  return gemv_rows<8, T>(X, M, K, qw, qz, sc, gi, xp, G, N, Y, s);
 }
 
 int check_qlinear(const int32_t* qweight, const int32_t* qzeros, const uint16_t* scales, const int32_t* g_idx,
@@ -697,30 +803,74 @@ extern "C" int gptq_dequantize_weight(const int32_t* qweight, const int32_t* qze
 
 extern "C" int gptq_quantized_linear(const void* X, int x_dtype, int64_t M, int64_t n_in, const int32_t* qweight,
                                      const int32_t* qzeros, const uint16_t* scales_f16, const int32_t* g_idx,
-                                     int64_t groups, int64_t n_out, int bits, void* Y, void* stream) {
+                                     const int32_t* x_perm, int64_t groups, int64_t n_out, int bits, void* Y,
+                                     void* stream) {
   GPTQ_TRY(check_qlinear(qweight, qzeros, scales_f16, g_idx, groups, n_in, n_out, bits));
   if (M < 0 || ((!X || !Y) && M > 0)) return GPTQ_ERR_INVALID_ARG;  // no rows: X and Y may be NULL
   if (x_dtype != GPTQ_F16 && x_dtype != GPTQ_BF16) return GPTQ_ERR_INVALID_ARG;
   if (M == 0) return GPTQ_OK;
   if (M >= (int64_t(1) << 31)) return GPTQ_ERR_UNSUPPORTED;
-  if (!aligned16(X) || !aligned16(Y)) return GPTQ_ERR_UNSUPPORTED;
+  if (!aligned16(X) || !aligned16(Y) || (x_perm && !aligned16(x_perm))) return GPTQ_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const __half* sc = reinterpret_cast<const __half*>(scales_f16);
   const int G = static_cast<int>(groups);
   if (M <= GV_MAXM) {
     if (x_dtype == GPTQ_BF16)
       return gemv_any<__nv_bfloat16>(bits, static_cast<const __nv_bfloat16*>(X), static_cast<int>(M), n_in, qweight,
-                                     qzeros, sc, g_idx, G, n_out, static_cast<__nv_bfloat16*>(Y), s);
+                                     qzeros, sc, g_idx, x_perm, G, n_out, static_cast<__nv_bfloat16*>(Y), s);
     return gemv_any<__half>(bits, static_cast<const __half*>(X), static_cast<int>(M), n_in, qweight, qzeros, sc, g_idx,
-                            G, n_out, static_cast<__half*>(Y), s);
+                            x_perm, G, n_out, static_cast<__half*>(Y), s);
   }
+  const size_t xbytes = x_perm ? static_cast<size_t>(M) * n_in * 2 : 0;
   void* Wd = nullptr;
-  GPTQ_TRY(pool_alloc(&Wd, static_cast<size_t>(n_in) * n_out * 2, s));
-  int st = x_dtype == GPTQ_BF16
-               ? dequant_any<__nv_bfloat16>(bits, qweight, qzeros, sc, g_idx, G, n_in, n_out,
-                                            static_cast<__nv_bfloat16*>(Wd), s)
-               : dequant_any<__half>(bits, qweight, qzeros, sc, g_idx, G, n_in, n_out, static_cast<__half*>(Wd), s);
-  if (st == GPTQ_OK) st = gemm_bf16_tn(X, Wd, Y, M, n_out, n_in, x_dtype, s);
+  GPTQ_TRY(pool_alloc(&Wd, static_cast<size_t>(n_in) * n_out * 2 + xbytes, s));
+  const void* Xg = X;
+  int st = GPTQ_OK;
+  if (x_perm) {  // X with its columns in the order of the codes
+    void* Xp = static_cast<char*>(Wd) + static_cast<size_t>(n_in) * n_out * 2;
+    const int64_t cnt = M * n_in;
+    const unsigned gx = static_cast<unsigned>((cnt + 255) / 256);
+    if (x_dtype == GPTQ_BF16)
+      gather_cols_kernel<__nv_bfloat16><<<gx, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(X), x_perm, M, n_in,
+                                                           static_cast<__nv_bfloat16*>(Xp));
+    else
+      gather_cols_kernel<__half><<<gx, 256, 0, s>>>(static_cast<const __half*>(X), x_perm, M, n_in,
+                                                    static_cast<__half*>(Xp));
+    st = after_launch();
+    Xg = Xp;
+  }
+  if (st == GPTQ_OK)
+    st = x_dtype == GPTQ_BF16
+             ? dequant_any<__nv_bfloat16>(bits, qweight, qzeros, sc, g_idx, G, n_in, n_out,
+                                          static_cast<__nv_bfloat16*>(Wd), s)
+             : dequant_any<__half>(bits, qweight, qzeros, sc, g_idx, G, n_in, n_out, static_cast<__half*>(Wd), s);
+  if (st == GPTQ_OK) st = gemm_bf16_tn(Xg, Wd, Y, M, n_out, n_in, x_dtype, s);
   pool_free(Wd, s);
   return st;
+}
+
+extern "C" int gptq_reorder_act_order(const int32_t* qweight, const int32_t* g_idx, int64_t groups, int64_t n_in,
+                                      int64_t n_out, int bits, int32_t* qweight_out, int32_t* g_idx_out,
+                                      int32_t* x_perm, void* stream) {
+  if (!qweight || !g_idx || !qweight_out || !g_idx_out || !x_perm) return GPTQ_ERR_INVALID_ARG;
+  if (n_in <= 0 || n_out <= 0 || groups <= 0) return GPTQ_ERR_INVALID_ARG;
+  if (bits != 2 && bits != 3 && bits != 4 && bits != 8) return GPTQ_ERR_INVALID_ARG;
+  if (bits == 3) return GPTQ_ERR_UNSUPPORTED;
+  if (n_in % 64 != 0 || groups > n_in || n_in > 65536 || n_out > (int64_t(1) << 30)) return GPTQ_ERR_UNSUPPORTED;
+  if (qweight == qweight_out || g_idx == g_idx_out) return GPTQ_ERR_INVALID_ARG;  // not in place
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int G = static_cast<int>(groups), K = static_cast<int>(n_in);
+  const int smem = (G + 2 * RO_THREADS) * static_cast<int>(sizeof(int));
+  GPTQ_TRY(ensure_smem_limit(reinterpret_cast<const void*>(sort_by_group_kernel), smem));
+  sort_by_group_kernel<<<1, RO_THREADS, smem, s>>>(g_idx, K, G, x_perm, g_idx_out);
+  GPTQ_TRY(after_launch());
+  const int64_t rows = n_in * bits / 32;
+  const dim3 grid(static_cast<unsigned>((n_out + 255) / 256), static_cast<unsigned>(rows));
+  if (bits == 2)
+    reorder_codes_kernel<2><<<grid, 256, 0, s>>>(qweight, x_perm, rows, n_out, qweight_out);
+  else if (bits == 4)
+    reorder_codes_kernel<4><<<grid, 256, 0, s>>>(qweight, x_perm, rows, n_out, qweight_out);
+  else
+    reorder_codes_kernel<8><<<grid, 256, 0, s>>>(qweight, x_perm, rows, n_out, qweight_out);
+  return after_launch();
 }

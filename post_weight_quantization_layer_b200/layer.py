@@ -24,15 +24,25 @@ from . import api
 
 @dataclass
 class LayerTimes:
-    hessian_ms: float = 0.0
+    hessian_ms: float = 0.0  # start until every Hessian is accumulated
     factor_ms: float = 0.0  # two-phase route only
     sweep_ms: float = 0.0  # two-phase route only
-    factor_sweep_ms: float = 0.0  # factors and sweeps together (both routes)
+    # two-phase: factors and sweeps; pipelined: from the largest Hessian's completion (where
+    # its factor starts) to the end, overlapping the other Hessians' accumulation
+    factor_sweep_ms: float = 0.0
+    total_ms: float = 0.0
     hessian_launch_ms: list = field(default_factory=list)
 
-    @property
-    def total_ms(self):
-        return self.hessian_ms + self.factor_sweep_ms
+
+_side_streams = {}
+
+
+def _side_stream(device):
+    """A library-side torch stream per device for the smaller Hessians of a pipelined layer."""
+    key = torch.device(device).index
+    if key not in _side_streams:
+        _side_streams[key] = torch.cuda.Stream(device=device)
+    return _side_streams[key]
 
 
 def quantize_decoder_layer(acts, weights, modules, qcfg, hessians=None, timing=False, stream=None,
@@ -55,34 +65,68 @@ def quantize_decoder_layer(acts, weights, modules, qcfg, hessians=None, timing=F
     times = LayerTimes() if timing else None
     marks = []
 
-    def mark():
+    def mark_on(st):
         if timing:
             e = ev()
-            e.record(stream)
+            e.record(st)
             marks.append(e)
             return e
         return None
 
+    def mark():
+        return mark_on(stream)
+
     with torch.cuda.stream(stream):
-        mark()
+        m0 = mark()
         Hs = {}
         launch_marks = []
+        ready = None
+        m_first = None
         if hessians_given:
             if not hessians:
                 raise ValueError("hessians_given needs the layer's Hessians in `hessians`")
             Hs = dict(hessians)
-        for h, X in ({} if hessians_given else acts).items():
-            chunks = X if isinstance(X, (list, tuple)) else [X]
-            n = chunks[0].shape[1]
-            H = hessians[h] if hessians is not None else torch.empty(n, n, dtype=torch.float32, device=chunks[0].device)
-            H.zero_()
-            a = mark()
-            for c in chunks:
-                api.accumulate_hessian(c, H, stream=stream)
-            b = mark()
-            launch_marks.append((a, b))
-            Hs[h] = H
-        m_h = mark()
+        else:
+            def width(X):
+                return (X[0] if isinstance(X, (list, tuple)) else X).shape[1]
+
+            for h, X in acts.items():
+                n = width(X)
+                chunks = X if isinstance(X, (list, tuple)) else [X]
+                Hs[h] = hessians[h] if hessians is not None else torch.empty(n, n, dtype=torch.float32,
+                                                                             device=chunks[0].device)
+
+            def accumulate(h, st):
+                X = acts[h]
+                chunks = X if isinstance(X, (list, tuple)) else [X]
+                with torch.cuda.stream(st):
+                    Hs[h].zero_()
+                    a = mark_on(st)
+                    for c in chunks:
+                        api.accumulate_hessian(c, Hs[h], stream=st)
+                    launch_marks.append((h, a, mark_on(st)))
+
+            # the largest Hessian first: with the pipelined route its factor (the layer's
+            # critical path) starts while the others are still being accumulated
+            order = sorted(acts, key=lambda h: -width(acts[h]))
+            accumulate(order[0], stream)
+            m_first = mark()
+            if pipelined and len(order) > 1:
+                side = _side_stream(stream.device)
+                side.wait_stream(stream)
+                for h in order[1:]:
+                    accumulate(h, side)
+                side_done = torch.cuda.Event(enable_timing=timing)
+                side_done.record(side)
+                ready = [None if h == order[0] else side_done for h in Hs]
+                m_h = side_done if timing else None
+            else:
+                for h in order[1:]:
+                    accumulate(h, stream)
+        if ready is None:
+            m_h = mark()
+        if m_first is None:
+            m_first = m_h
         keys = list(Hs)
         m_f = None
         if pipelined:
@@ -90,7 +134,7 @@ def quantize_decoder_layer(acts, weights, modules, qcfg, hessians=None, timing=F
             mods = list(modules)
             _, res = api.quantize_linears([Hs[h] for h in keys], [(weights[m.name], hpos[m.h_index]) for m in mods],
                                           qcfg.bits, qcfg.group_size, qcfg.damp_percent, qcfg.sym, qcfg.desc_act,
-                                          qcfg.static_groups, qcfg.blocksize, stream=stream)
+                                          qcfg.static_groups, qcfg.blocksize, stream=stream, ready=ready)
             results = {m.name: r for m, r in zip(mods, res)}
         else:
             # every distinct Hessian factored in one call: the library runs them concurrently
@@ -106,10 +150,12 @@ def quantize_decoder_layer(acts, weights, modules, qcfg, hessians=None, timing=F
         m_s = mark()
     if timing:
         m_s.synchronize()
-        times.hessian_ms = marks[0].elapsed_time(m_h)
-        times.factor_sweep_ms = m_h.elapsed_time(m_s)
+        times.hessian_ms = m0.elapsed_time(m_h)
+        times.factor_sweep_ms = (m_h if ready is None else m_first).elapsed_time(m_s)
+        times.total_ms = m0.elapsed_time(m_s)
         if m_f is not None:
             times.factor_ms = m_h.elapsed_time(m_f)
             times.sweep_ms = m_f.elapsed_time(m_s)
-        times.hessian_launch_ms = [a.elapsed_time(b) for a, b in launch_marks]
+        by_h = {h: a.elapsed_time(b) for h, a, b in launch_marks}
+        times.hessian_launch_ms = [by_h[h] for h in sorted(by_h)]
     return results, times

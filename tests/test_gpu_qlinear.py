@@ -115,3 +115,43 @@ def test_linear_zero_rows_and_determinism():
     torch.cuda.synchronize()
     assert torch.equal(a, b) and torch.equal(c, d)
     assert gq.device_status() == 0
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("bits,g", [(4, 128), (2, 32), (8, 64)])
+@pytest.mark.parametrize("M", [1, 3, 130])
+def test_reordered_act_order_checkpoint(dtype, bits, g, M):
+    """gptq_reorder_act_order: the inputs sorted stably by (g_idx, index), the codes and g_idx
+    carried along (index work: exact); the dequantized weight is the original's columns in that
+    order (bit-exact); the linear on it is the same product (same bound) on both paths."""
+    n_out, n_in = 272, 1024
+    ck, W = _checkpoint(n_out, n_in, bits, g, 40 + bits + M, True)
+    ck2 = gq.reorder_act_order(ck, bits)
+    torch.cuda.synchronize()
+    gi = ck["g_idx"].cpu().numpy()
+    xp = ck2["x_perm"].cpu().numpy()
+    assert np.array_equal(xp, np.lexsort((np.arange(n_in), gi)))
+    assert np.array_equal(ck2["g_idx"].cpu().numpy(), gi[xp])
+    assert np.all(np.diff(ck2["g_idx"].cpu().numpy()) >= 0)
+    W16 = O.round16(W, NAME[dtype])
+    Wd = gq.dequantize_weight(ck2, bits, dtype)
+    torch.cuda.synchronize()
+    assert np.array_equal(Wd.double().cpu().numpy(), W16[:, xp])
+    X = synth.StudentTActs(n_in, M, 70 + M, dtype=dtype).full()
+    Y = gq.quantized_linear(X.to(device()), ck2, bits)
+    torch.cuda.synchronize()
+    _tol_check(Y, X, W16, dtype)
+
+
+def test_reordered_checkpoint_llama_decode():
+    """A Llama-shaped act-order checkpoint (4096 -> 11008): the reordered decode agrees with the
+    original checkpoint's decode within the fp32 accumulation bound."""
+    dtype = torch.bfloat16
+    ck, W = _checkpoint(11008, 4096, 4, 128, 91, True)
+    ck2 = gq.reorder_act_order(ck, 4)
+    X = synth.StudentTActs(4096, 1, 92, dtype=dtype).full()
+    Y = gq.quantized_linear(X.to(device()), ck2, 4)
+    torch.cuda.synchronize()
+    _tol_check(Y, X, O.round16(W, "bfloat16"), dtype)
+    with pytest.raises(ValueError):
+        gq.reorder_act_order(ck2, 4)

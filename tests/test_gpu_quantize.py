@@ -193,3 +193,34 @@ def test_pipelined_linears_report_the_failing_linear():
     U1, p1 = gq.factor_hessian(good, 0.01, True)
     b = gq.quantize_layer_factored(lin[0][0], U1, p1, 4, 32, True, False, 128)
     assert torch.equal(res[0].qweight, b.qweight)
+
+
+@pytest.mark.parametrize("cfgname", ["opt125m", "llama7b"])
+def test_layer_driver_routes_agree(cfgname):
+    """The layer driver's pipelined route (the largest Hessian accumulated first, its factor
+    started while the others accumulate on a side stream, every sweep on its own stream)
+    against the two-phase route on the very Hessians the pipelined run accumulated: the same
+    codes, scales, zero points and g_idx, bit for bit."""
+    from post_weight_quantization_layer_b200.layer import quantize_decoder_layer
+    dev = device()
+    cfg = synth.CONFIGS[cfgname]
+    acts = {h: synth.acts_for(cfg, h, tokens=4096).full(device=dev) for h in range(len(cfg.hessian_n))}
+    weights = {m.name: synth.weight_for(cfg, m, device=dev) for m in cfg.layers}
+    Hbuf = {h: torch.empty(n, n, dtype=torch.float32, device=dev) for h, n in enumerate(cfg.hessian_n)}
+    a, ta = quantize_decoder_layer(acts, weights, cfg.layers, cfg, hessians=Hbuf, timing=True, pipelined=True)
+    torch.cuda.synchronize()
+    given = {h: H.clone() for h, H in Hbuf.items()}
+    b, tb = quantize_decoder_layer(None, weights, cfg.layers, cfg, hessians=given, timing=True,
+                                   hessians_given=True, pipelined=False)
+    torch.cuda.synchronize()
+    for m in cfg.layers:
+        ra, rb = a[m.name], b[m.name]
+        for x, y in zip((ra.qweight, ra.scales, ra.zeros, ra.g_idx), (rb.qweight, rb.scales, rb.zeros, rb.g_idx)):
+            assert torch.equal(x, y), m.name
+    for h, X in acts.items():
+        # every Hessian was accumulated (the largest on the caller's stream, the rest on the
+        # side stream): its leading 64 x 64 block against the oracle
+        ref = O.hessian(X[:, :64].double().cpu().numpy())
+        got = Hbuf[h][:64, :64].double().cpu().numpy()
+        assert np.abs(got - ref).max() <= 1e-5 * np.abs(ref).max(), h
+    assert ta.total_ms > 0 and tb.total_ms > 0 and tb.factor_ms > 0 and tb.sweep_ms > 0

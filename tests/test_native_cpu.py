@@ -18,6 +18,7 @@ from tests.conftest import read_golden
 INVALID, UNSUPPORTED = 1, 2
 FAKE = ctypes.c_void_p(0x10000)
 MISALIGNED = ctypes.c_void_p(0x10004)
+FAKE2 = ctypes.c_void_p(0x20000)  # a second distinct (never dereferenced) pointer
 
 
 @pytest.fixture(scope="module")
@@ -180,12 +181,19 @@ def test_checkpoint_and_forward_rejections(L):
     assert dq(FAKE, FAKE, FAKE, FAKE, 4, 512, 72, 2, 1, FAKE, None) == UNSUPPORTED   # 72*2 % 32
     assert dq(FAKE, FAKE, FAKE, FAKE, 4, 512, 64, 4, 0, FAKE, None) == INVALID       # fp32 output
     ql = L.gptq_quantized_linear
-    assert ql(FAKE, 2, 8, 512, FAKE, FAKE, FAKE, FAKE, 4, 64, 4, None, None) == INVALID
-    assert ql(FAKE, 0, 8, 512, FAKE, FAKE, FAKE, FAKE, 4, 64, 4, FAKE, None) == INVALID   # fp32 X
-    assert ql(FAKE, 2, -1, 512, FAKE, FAKE, FAKE, FAKE, 4, 64, 4, FAKE, None) == INVALID
-    assert ql(FAKE, 2, 0, 512, FAKE, FAKE, FAKE, FAKE, 4, 64, 4, FAKE, None) == 0         # no rows: no-op
-    assert ql(None, 2, 0, 512, FAKE, FAKE, FAKE, FAKE, 4, 64, 4, None, None) == 0         # ... even with NULL X, Y
-    assert ql(MISALIGNED, 2, 8, 512, FAKE, FAKE, FAKE, FAKE, 4, 64, 4, FAKE, None) == UNSUPPORTED
+    assert ql(FAKE, 2, 8, 512, FAKE, FAKE, FAKE, FAKE, None, 4, 64, 4, None, None) == INVALID
+    assert ql(FAKE, 0, 8, 512, FAKE, FAKE, FAKE, FAKE, None, 4, 64, 4, FAKE, None) == INVALID   # fp32 X
+    assert ql(FAKE, 2, -1, 512, FAKE, FAKE, FAKE, FAKE, None, 4, 64, 4, FAKE, None) == INVALID
+    assert ql(FAKE, 2, 0, 512, FAKE, FAKE, FAKE, FAKE, None, 4, 64, 4, FAKE, None) == 0         # no rows: no-op
+    assert ql(None, 2, 0, 512, FAKE, FAKE, FAKE, FAKE, None, 4, 64, 4, None, None) == 0         # ... even NULL X, Y
+    assert ql(MISALIGNED, 2, 8, 512, FAKE, FAKE, FAKE, FAKE, None, 4, 64, 4, FAKE, None) == UNSUPPORTED
+    assert ql(FAKE, 2, 8, 512, FAKE, FAKE, FAKE, FAKE, MISALIGNED, 4, 64, 4, FAKE, None) == UNSUPPORTED
+    ro = L.gptq_reorder_act_order
+    assert ro(None, FAKE, 4, 512, 64, 4, FAKE2, FAKE2, FAKE2, None) == INVALID
+    assert ro(FAKE, FAKE, 4, 512, 64, 5, FAKE2, FAKE2, FAKE2, None) == INVALID
+    assert ro(FAKE, FAKE, 4, 512, 64, 3, FAKE2, FAKE2, FAKE2, None) == UNSUPPORTED   # 3-bit
+    assert ro(FAKE, FAKE, 4, 500, 64, 4, FAKE2, FAKE2, FAKE2, None) == UNSUPPORTED   # n_in % 64
+    assert ro(FAKE, FAKE, 4, 512, 64, 4, FAKE, FAKE2, FAKE2, None) == INVALID        # in place
     assert L.gptq_rmsnorm(FAKE, 0, 4, 64, FAKE, 1e-6, FAKE, None) == INVALID
     assert L.gptq_rmsnorm(FAKE, 2, 4, 64, None, 1e-6, FAKE, None) == INVALID
     assert L.gptq_rope(FAKE, 2, 16, 4, 63, 8, 10000.0, None) == INVALID   # odd head_dim
