@@ -293,6 +293,9 @@ def run_native(args, world, rank, local):
         "traffic": None,
         "algorithmic_flops_per_launch": work["hessian_flops"],
         "per_launch_tflops": [round(x, 1) for x in per_launch],
+        "launch_timing": ("the timed steps' launches" if args.two_phase else
+                          "launches of the two-phase steps after the timed region (in the pipelined steps "
+                          "three of the four Hessians overlap the largest one's factorisation)"),
     }
     traffic = hessian_traffic(cfg, T)
     if traffic is not None:

@@ -159,7 +159,7 @@ int sweep_common(const void* W, int w_dtype, int64_t n_out, int64_t n_in, const 
                  const int32_t* invperm, int bits, int group_size, int sym, int static_groups, int blocksize,
                  int32_t* qweight, float* scales, int32_t* zeros, int32_t* g_idx, double* Wk, double* Err,
                  uint8_t* codesT, double* loss, int* status, cudaStream_t s, gptq_stats* stats, Events& evs,
-                 int ev0) {
+                 int ev0, bool low_priority = false) {
   SweepArgs a;
   a.W = W;
   a.w_dtype = w_dtype;
@@ -184,6 +184,7 @@ int sweep_common(const void* W, int w_dtype, int64_t n_out, int64_t n_in, const 
   a.status = status;
   a.stats = stats;
   for (int i = 0; i < 4; ++i) a.ev[i] = evs.on ? evs.ev[ev0 + i] : nullptr;
+  a.low_priority = low_priority ? 1 : 0;
   int pw = 0, qw = 0;
   GPTQ_TRY(run_sweep(a, s, &pw, &qw));
   if (stats) {
@@ -442,7 +443,8 @@ int gptq_quantize_linears(int n_hessians, const float* const* H, const int64_t* 
         GPTQ_TRY(sweep_common(W[j], w_dtype, n_out[j], ni, U[i], desc_act ? perm[i] : nullptr,
                               desc_act ? invperm[static_cast<size_t>(i)] : nullptr, bits, group_size, sym,
                               static_groups, blocksize, qweight[j], scales[j], zeros[j], g_idx[j], Wk, Err, codesT,
-                              loss, dstat + n_hessians + j, lease[static_cast<int>(t)].st, nullptr, off, 0));
+                              loss, dstat + n_hessians + j, lease[static_cast<int>(t)].st, nullptr, off, 0,
+                              /*low_priority: the largest Hessian's sweeps follow the critical path*/ i != largest));
       }
     }
   }  // every lane joins back into s

@@ -140,6 +140,7 @@ struct SweepArgs {
   int* status;
   gptq_stats* stats;      // may be null
   cudaEvent_t ev[4];      // valid when stats != null
+  int low_priority = 0;   // panels and look-ahead on a low-priority lane too
 };
 int run_sweep(SweepArgs& a, cudaStream_t s, int* panel_width, int* outer_width);
 

@@ -601,7 +601,9 @@ int run_sweep(SweepArgs& a, cudaStream_t s, int* panel_width, int* outer_width) 
 
   {
     LaneLease lanes(s);
-    const LanePrio prio[2] = {kLaneHigh, kLaneLow};  // panels + look-ahead; trailing update
+    // panels + look-ahead (high, unless the caller runs this sweep beside more urgent work);
+    // trailing update
+    const LanePrio prio[2] = {a.low_priority ? kLaneLow : kLaneHigh, kLaneLow};
     GPTQ_TRY(lanes.acquire(2, prio));
     cudaStream_t sp = lanes[0].st, sg = lanes[1].st;
     cudaEvent_t pan = lanes[0].aux, rest = lanes[1].aux;
