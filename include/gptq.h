@@ -305,8 +305,8 @@ int gptq_quantized_linear(const void* X, int x_dtype, int64_t M, int64_t n_in, c
  * fp32 sums taken in another order; gptq_dequantize_weight on it gives W_hat[:, x_perm].
  * qweight [n_in*bits/32, n_out] and g_idx [n_in] read-only; qweight_out (same shape),
  * g_idx_out and x_perm ([n_in] int32) written, none aliasing an input.  g_idx entries outside
- * [0, groups) are clamped.  bits 2, 4, 8 (3 -> UNSUPPORTED); n_in % 64 == 0 and n_in <= 65536,
- * else UNSUPPORTED.  Asynchronous on `stream`; the sort runs in one CTA (a preparation
+ * [0, groups) are clamped.  bits 2, 4, 8 (3 -> UNSUPPORTED); n_in % 64 == 0, n_in <= 65536
+ * and groups <= 32768, else UNSUPPORTED.  Asynchronous on `stream`; the sort runs in one CTA (a preparation
  * step, once per checkpoint).
  */
 int gptq_reorder_act_order(const int32_t* qweight, const int32_t* g_idx, int64_t groups, int64_t n_in,

@@ -856,7 +856,9 @@ extern "C" int gptq_reorder_act_order(const int32_t* qweight, const int32_t* g_i
   if (n_in <= 0 || n_out <= 0 || groups <= 0) return GPTQ_ERR_INVALID_ARG;
   if (bits != 2 && bits != 3 && bits != 4 && bits != 8) return GPTQ_ERR_INVALID_ARG;
   if (bits == 3) return GPTQ_ERR_UNSUPPORTED;
-  if (n_in % 64 != 0 || groups > n_in || n_in > 65536 || n_out > (int64_t(1) << 30)) return GPTQ_ERR_UNSUPPORTED;
+  // the group counters live in shared memory: at most 32768 groups
+  if (n_in % 64 != 0 || groups > n_in || groups > 32768 || n_in > 65536 || n_out > (int64_t(1) << 30))
+    return GPTQ_ERR_UNSUPPORTED;
   if (qweight == qweight_out || g_idx == g_idx_out) return GPTQ_ERR_INVALID_ARG;  // not in place
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int G = static_cast<int>(groups), K = static_cast<int>(n_in);

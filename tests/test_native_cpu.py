@@ -194,6 +194,7 @@ def test_checkpoint_and_forward_rejections(L):
     assert ro(FAKE, FAKE, 4, 512, 64, 3, FAKE2, FAKE2, FAKE2, None) == UNSUPPORTED   # 3-bit
     assert ro(FAKE, FAKE, 4, 500, 64, 4, FAKE2, FAKE2, FAKE2, None) == UNSUPPORTED   # n_in % 64
     assert ro(FAKE, FAKE, 4, 512, 64, 4, FAKE, FAKE2, FAKE2, None) == INVALID        # in place
+    assert ro(FAKE, FAKE, 40000, 65536, 64, 4, FAKE2, FAKE2, FAKE2, None) == UNSUPPORTED  # > 32768 groups
     assert L.gptq_rmsnorm(FAKE, 0, 4, 64, FAKE, 1e-6, FAKE, None) == INVALID
     assert L.gptq_rmsnorm(FAKE, 2, 4, 64, None, 1e-6, FAKE, None) == INVALID
     assert L.gptq_rope(FAKE, 2, 16, 4, 63, 8, 10000.0, None) == INVALID   # odd head_dim
