@@ -421,8 +421,8 @@ __global__ void __maxnreg__(160)
     // owns one column n (its TMEM lane); the 4 warps of each lane quarter are split over the
     // tile's BN rows in chunks of CR (warps 2..5 take the even chunks, 6..9 the odd ones); for
     // each row the warp's 32 lanes update 32 consecutive columns (coalesced).  The CR loads of
-    // C are issued together before any use, and the rows of this CTA's next tile are
-    // prefetched into L2 while the current one is updated.
+    // C are issued together, before the accumulator reads, and the rows of this CTA's next tile
+    // are prefetched into L2 while the current one is updated.
     const int quad = warp & 3;
     const int half = (warp - 2) >> 2;
     const int et = threadIdx.x - 64;  // 0..255 over the epilogue warps
@@ -460,16 +460,17 @@ __global__ void __maxnreg__(160)
       const int ec = cin ? a.eb[a.col0 + c] - 2 * SBETA - 3 * SBETA : 0;
       for (int chunk = half; chunk < BN / CR; chunk += 2) {
         const int r0 = t.r0 + chunk * CR;
+        // the C loads first, so that their latency overlaps the accumulator reads
+        double cv[CR];
+#pragma unroll
+        for (int j = 0; j < CR; ++j)
+          cv[j] = (cin && r0 + j < a.M) ? a.C[static_cast<int64_t>(r0 + j) * a.ldc + c] : 0.0;
         int acc[NS][CR];
 #pragma unroll
         for (int s = 0; s < NS; ++s)
           tmem_ld_32x32b(tmem + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(b * NS * BN + s * BN + chunk * CR),
                          acc[s]);
-        double cv[CR];
-#pragma unroll
-        for (int j = 0; j < CR; ++j)
-          cv[j] = (cin && r0 + j < a.M) ? a.C[static_cast<int64_t>(r0 + j) * a.ldc + c] : 0.0;
 #pragma unroll
         for (int j = 0; j < CR; ++j) {
           long long hi = acc[0][j];
