@@ -203,3 +203,58 @@ def test_checkpoint_and_forward_rejections(L):
     assert L.gptq_silu_mul(FAKE, None, 2, 8, FAKE, None) == INVALID
     assert L.gptq_add(FAKE, FAKE, 1, -1, FAKE, None) == INVALID
     assert L.gptq_test_wait_expiry(1, 0) == INVALID
+
+
+def test_pipelined_linears_rejections(L):
+    """gptq_quantize_linears rejects bad arguments before any device work."""
+    f = L.gptq_quantize_linears
+    P2 = ctypes.c_void_p * 2
+    hp = P2(FAKE, FAKE)
+    ns = (ctypes.c_int64 * 2)(256, 512)
+    wp = P2(FAKE, FAKE)
+    no = (ctypes.c_int64 * 2)(64, 64)
+    hof = (ctypes.c_int * 2)(0, 1)
+    st = (ctypes.c_int * 2)()
+
+    def call(nh=2, H=hp, n_in=ns, damp=0.01, nl=2, W=wp, n_out=no, hidx=hof, bits=4, g=128, bs=128):
+        return f(nh, H, n_in, damp, 1, hp, hp, nl, W, 1, n_out, hidx, bits, g, 1, 0, bs, wp, wp, wp, wp, None, None,
+                 st)
+    assert call(nh=0) == INVALID
+    assert call(nl=0) == INVALID
+    assert call(H=None) == INVALID
+    assert call(damp=0.0) == INVALID
+    assert call(damp=math.nan) == INVALID
+    assert call(hidx=(ctypes.c_int * 2)(0, 2)) == INVALID                     # Hessian index out of range
+    assert call(hidx=(ctypes.c_int * 2)(0, -1)) == INVALID
+    assert call(n_in=(ctypes.c_int64 * 2)(256, 500)) == UNSUPPORTED           # n_in % 8
+    assert call(bits=5) == INVALID                                            # a config rule per linear
+    assert call(H=P2(FAKE, MISALIGNED)) == UNSUPPORTED
+    assert call(W=P2(FAKE, None)) == INVALID
+
+
+def test_pipelined_and_reorder_binding_rejections():
+    import torch
+
+    import post_weight_quantization_layer_b200 as gq
+    H = torch.zeros(64, 64)
+    W = torch.zeros(8, 64, dtype=torch.float16)
+    ck = {"qweight": torch.zeros(8, 16, dtype=torch.int32), "qzeros": torch.zeros(1, 2, dtype=torch.int32),
+          "scales": torch.zeros(1, 16, dtype=torch.float16), "g_idx": torch.zeros(64, dtype=torch.int32)}
+    cases = [
+        (lambda: gq.quantize_linears([], [(W, 0)]), "at least one"),
+        (lambda: gq.quantize_linears([H], []), "at least one"),
+        (lambda: gq.quantize_linears([H], [(W, 1)]), "out of range"),
+        (lambda: gq.quantize_linears([H], [(torch.zeros(8, 32, dtype=torch.float16), 0)]), "does not match"),
+        (lambda: gq.quantize_linears([H], [(W, 0), (W.float(), 0)]), "same weight dtype"),
+        (lambda: gq.quantize_linears([H.half()], [(W, 0)]), r"H\[0\] must have dtype"),
+        (lambda: gq.quantize_linears([H], [(W, 0)], ready=[None, None]), "one entry"),
+        (lambda: gq.quantize_linears([H], [(W, 0)]), "CUDA tensors"),
+        (lambda: gq.reorder_act_order(dict(ck, x_perm=torch.zeros(64, dtype=torch.int32))), "already reordered"),
+        (lambda: gq.reorder_act_order(dict(ck, x_perm=torch.zeros(32, dtype=torch.int32))), "x_perm must have shape"),
+        (lambda: gq.quantized_linear(torch.zeros(1, 64, dtype=torch.float16),
+                                     dict(ck, x_perm=torch.zeros(64, dtype=torch.int64))), "x_perm must have dtype"),
+        (lambda: gq.reorder_act_order(ck), "CUDA tensors"),
+    ]
+    for fn, msg in cases:
+        with pytest.raises(ValueError, match=msg):
+            fn()
