@@ -20,13 +20,15 @@
 //   U11 = factor-and-invert(A'),  U12 = -U11 T,
 // since V^-1 = [[V11^-1, -V11^-1 V12 V22^-1], [0, V22^-1]].  Blocks of at most NB = 128 are
 // factored and inverted by one CTA in shared memory (which also checks every pivot);
-// everything else is four large GEMMs per level.  V itself is never stored.
+// everything else is four large products per level: on the fp64 matrix units for nodes whose
+// right part is narrower than 1024, on the int8 tensor cores (seven-slice operands, exact
+// integer slice products, ozaki.cu) above.  V itself is never stored.
 //
-// Precision: the factorisation runs in fp64 and U stays fp64.  The forward error of a
-// Cholesky factor grows like cond(H_d) times the working precision; with cond(H_d) ~ 1e4
-// (heavy-tailed activation channels) an fp32 factorisation leaves ~1e-5 relative error
-// in U, and a sweep over thousands of columns amplifies even fp32 rounding of U into
-// different codes.
+// Precision: the factorisation runs in fp64 (the int8 route carries 49 bits of every operand
+// and adds exact integer products) and U stays fp64.  The forward error of a Cholesky factor
+// grows like cond(H_d) times the working precision; with cond(H_d) ~ 1e4 (heavy-tailed
+// activation channels) an fp32 factorisation leaves ~1e-5 relative error in U, and a sweep
+// over thousands of columns amplifies even fp32 rounding of U into different codes.
 #include <algorithm>
 #include <vector>
 
