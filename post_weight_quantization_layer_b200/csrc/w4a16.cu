@@ -23,6 +23,10 @@
 //   tensor cores: TMA loads of both K-major operands with 128-byte swizzle into a 4-stage
 //   ring, tcgen05.mma kind::f16 into a TMEM accumulator of 128 x 256, persistent CTAs with
 //   two accumulators in TMEM so that one tile's epilogue overlaps the next tile's MMAs.
+// An act-order checkpoint (g_idx not in order) can be reordered once (sort_by_group_kernel,
+// reorder_codes_kernel): its inputs sorted by group, with the permutation kept so that both
+// regimes read X in the same order (the decode kernel while staging X, the tensor-core path
+// through one gather).
 #include <cuda.h>
 
 #include <algorithm>
