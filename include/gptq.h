@@ -124,8 +124,10 @@ int gptq_accumulate_hessian(const void* X, int x_dtype, int64_t tokens, int64_t 
  *   g_idx   [n_in] int32: group of each original input column.
  *   Dequantized weight: scales[g_idx[c], o] * (code[o, c] - zeros[g_idx[c], o]).
  * n_in*bits % 32 != 0 or n_in % 8 != 0 -> UNSUPPORTED.
- * Workspace (about 3*n_in^2*8 + n_out*n_in*17 bytes, plus 10*(n_out + n_in)*B bytes of
- * int8 operand slices for the lazy block updates, B = 256 or 512) is taken stream-ordered
+ * Workspace (about 3*n_in^2*8 bytes for the factor, plus about 4.6*n_in^2 bytes of int8
+ * operand slices when n_in >= 2048; n_out*n_in*17 bytes for the sweep, plus
+ * 10*(n_out + n_in)*B bytes of int8 operand slices for its lazy block updates, B = 256 or
+ * 512) is taken stream-ordered
  * from a library-owned pool that keeps it cached for later calls (OOM if that fails; see
  * gptq_trim_workspace).  The call is blocking: it synchronises
  * `stream` once at the end and returns NOT_PD if a pivot failed.
@@ -202,10 +204,10 @@ int gptq_quantize_layer_factored(const void* W, int w_dtype, int64_t n_out, int6
  *       static_groups, blocksize, w_dtype, damp_percent, desc_act: shared by all.
  * Every output is bit-identical to gptq_factor_hessians followed by one
  * gptq_quantize_layer_factored per linear (the same kernels in the same order per item).
- * Scheduling: each Hessian's factor runs on its own library-owned stream (the largest at
- * the highest priority) and each linear's sweep on its own stream, started as soon as its
- * Hessian's factor is done, so the smaller Hessians' sweeps run while the largest factor is
- * still in progress.  All streams fork from `stream` and join back into it.  Workspace
+ * Scheduling: each Hessian's factor runs on its own library-owned stream and each linear's
+ * sweep on its own stream, started as soon as its Hessian's factor is done, so the smaller
+ * Hessians' sweeps run while the largest factor is still in progress; the largest Hessian's
+ * factor and sweeps (the critical path) run at high stream priority, the others at low.  All streams fork from `stream` and join back into it.  Workspace
  * (stream-ordered, from the library's pool): the factor workspaces of all Hessians plus
  * 17 * n_out[j] * n_in bytes per linear, held until the call returns.
  * hessian_ready: optional host array of n_hessians CUDA event handles (cudaEvent_t), NULL
