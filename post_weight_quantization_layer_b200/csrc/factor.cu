@@ -33,11 +33,16 @@
 #include <vector>
 
 #include "common.cuh"
+#include "factor_plan.h"
 
 namespace gptq {
 namespace {
 
-constexpr int NB = 128;  // leaf block width of the factorisation
+using fplan::NB;  // leaf block width of the factorisation
+using fplan::node_i8;
+using fplan::pad64;
+using fplan::Plan;
+using fplan::right_part;
 constexpr int DIAG_THREADS = 512;
 constexpr int SP = NB + 4;      // pitch of the diagonal block in shared memory (fragment loads
 constexpr int TP = NB / 2 + 4;  // of m8n8k4 hit 16 distinct bank pairs when pitch = 4 mod 16)
@@ -292,51 +297,6 @@ __global__ void __launch_bounds__(DIAG_THREADS) chol_diag_kernel(const real* A, 
 constexpr int DIAG_SMEM = (NB * SP + (NB / 2) * TP + 2 * NB + (NB / 16) * 16 * 17) * static_cast<int>(sizeof(real));
 
 
-// Recursion plan: block [lo, hi) splits at hi - n2 with n2 = ceil(n/2) rounded up to a
-// multiple of NB; blocks of at most NB are leaves.
-int64_t right_part(int64_t n) {
-  const int64_t half = (n + 1) / 2;
-  return std::min<int64_t>(n - 1, ((half + NB - 1) / NB) * NB);
-}
-
-// Nodes whose right part is at least I8_MIN wide run their four products on the int8
-// tensor cores (seven-slice operands: 49 bits each, see ozaki.cu); smaller ones on the fp64
-// matrix units.  Both K of a node's products (n2 and n1) stay within the int8 kernel's 16384.
-constexpr int64_t I8_MIN = 1024;
-constexpr int64_t I8_MAX = 16384;
-bool node_i8(int64_t n2) { return n2 >= I8_MIN && n2 <= I8_MAX; }
-
-int64_t pad64(int64_t k) { return (k + 63) / 64 * 64; }
-
-struct Plan {
-  size_t pmax = 0;
-  std::vector<size_t> tmax;            // T per depth
-  std::vector<size_t> sx, sy, ex, ey;  // int8 slices (bytes) and exponents per depth
-};
-
-// Largest P (n1 x n2) over all nodes, and per recursion depth the largest T and int8 slice
-// buffers: X [KSF][n1][pad(n2)] (rows of B, then of P, then of U11), Y [KSF][n2][pad(n2)]
-// (rows of U22, then its columns, then the columns of T).
-void plan(int64_t n, int depth, Plan& pl) {
-  if (n <= NB) return;
-  const int64_t n2 = right_part(n), n1 = n - n2;
-  const size_t sz = static_cast<size_t>(n1) * n2;
-  pl.pmax = std::max(pl.pmax, sz);
-  const size_t d = static_cast<size_t>(depth);
-  for (auto* v : {&pl.tmax, &pl.sx, &pl.sy, &pl.ex, &pl.ey})
-    if (v->size() <= d) v->resize(d + 1, 0);
-  pl.tmax[d] = std::max(pl.tmax[d], sz);
-  if (node_i8(n2)) {
-    const size_t ks = static_cast<size_t>(i8f_slices());
-    pl.sx[d] = std::max(pl.sx[d], ks * n1 * pad64(n2));
-    pl.sy[d] = std::max(pl.sy[d], ks * n2 * pad64(n2));
-    pl.ex[d] = std::max(pl.ex[d], static_cast<size_t>(n1));
-    pl.ey[d] = std::max(pl.ey[d], static_cast<size_t>(n2));
-  }
-  plan(n2, depth + 1, pl);
-  plan(n1, depth + 1, pl);
-}
-
 struct Scratch {
   real* P;
   real* P0;  // the top level's own P when its T product overlaps the left recursion
@@ -347,7 +307,7 @@ struct Scratch {
 
 size_t scratch_elems(int64_t n, Scratch* out, real* base, bool overlap) {
   Plan pl;
-  plan(n, 0, pl);
+  fplan::plan(n, 0, pl, static_cast<size_t>(i8f_slices()));
   size_t off = 0;
   auto take = [&](size_t e) {
     real* p = base ? base + off : nullptr;

@@ -21,8 +21,8 @@ def _h(n, T, seed, dtype=torch.float16):
 @pytest.mark.parametrize("n,T", [(256, 512), (264, 2000), (1032, 4096), (2056, 4112), (3000, 6000)])
 @pytest.mark.parametrize("desc_act", [False, True])
 def test_factor_matches_oracle(n, T, desc_act):
-    """Orders from 2048 up take the int8 route (seven-slice products) for their top-level
-    products; 2056 and 3000 leave ragged tiles in every product."""
+    """Orders above 1792 take the int8 route (seven-slice products) for the nodes whose right
+    part is at least 1024 wide; 2056 and 3000 leave ragged tiles in every product."""
     H = _h(n, T, n + T)
     U, perm = gq.factor_hessian(H.to(device()), 0.01, desc_act)
     torch.cuda.synchronize()

@@ -18,3 +18,14 @@ def test_schedule_covers_every_tile_and_segment_once(tmp_path):
     subprocess.run(["g++", "-O2", "-std=c++17", "-I", CSRC, src, "-o", str(exe)], check=True)
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=300)
     assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout
+
+
+@pytest.mark.skipif(shutil.which("g++") is None, reason="needs a host C++ compiler")
+def test_factor_plan_reserves_every_nodes_scratch(tmp_path):
+    """Host logic of the factor's recursion plan (the header factor.cu includes): every node's
+    products fit the per-depth scratch, int8 nodes stay within the int8 kernel's K range."""
+    exe = tmp_path / "factor_plan_check"
+    src = os.path.join(ROOT, "tests", "factor_plan_check.cpp")
+    subprocess.run(["g++", "-O2", "-std=c++17", "-I", CSRC, src, "-o", str(exe)], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout
